@@ -1,0 +1,229 @@
+/*
+ * usp.h -- C ABI of libusp: the Ulysses sequence-parallel attention block on
+ * one B200 (sm_100a), with P sequence-parallel ranks held as P virtual-rank
+ * buffers in one device's memory.
+ *
+ * Conventions (every entry point):
+ *  - Returns an int status, USP_OK (0) on success. On failure nothing has been
+ *    launched, and usp_last_error_message() (thread-local) says why.
+ *  - Device buffers are passed as plain device pointers and are owned by the
+ *    caller; the library never frees them. The library owns only the plan
+ *    (a host object plus one auxiliary CUDA stream and its events).
+ *  - "Per-rank arrays" are host arrays of `world` device pointers, element r
+ *    for virtual rank r; multi-tensor calls pass ntensors*world pointers,
+ *    tensor-major (all ranks of tensor 0, then tensor 1, ...).
+ *  - Every launch goes on the caller's stream (`stream`, a cudaStream_t; NULL
+ *    is the legacy default stream). No call synchronises the host, except
+ *    usp_device_status(). Calls are stream-ordered like any CUDA kernel.
+ *  - Tensors are dense and contiguous, row-major, in the BSHD layout of the
+ *    ragged transport page: [batch, tokens, heads, head_dim]. Pointers must be
+ *    16-byte aligned (USP_ERR_ALIGN otherwise); there is no slow path.
+ *  - Element types: USP_BF16, USP_FP16 (2 bytes) and USP_FP32 (4 bytes).
+ *    Layout operations copy bytes and are exact for any type.
+ *
+ * Notation: T = seq_len tokens split across ranks, prefix = replicated leading
+ * tokens (a cls token; 0 or 1), T' = prefix + T, H = heads, D = head_dim,
+ * B = batch, P = world. Rank r owns tokens [t0_r, t0_r + T_r) and heads
+ * [h0_r, h0_r + H_r), both from the balanced split (earlier ranks take the
+ * remainder). A sequence shard of rank r is [B, prefix + T_r, H, D]; a head
+ * shard of rank r is [B, T', H_r, D].
+ *
+ * Sources: "mstar.model.components.distributed.sequence_parallel" (API page),
+ * "h3_blackwell_runtime/distributed.py -- Ragged Ulysses sequence-parallel
+ * transport", "maxdiffusion PR #428: experimental two-phase (head-chunked)
+ * Ulysses all-to-all", "deepspeed/sequence/autosp_vit.py".
+ */
+#ifndef USP_H_
+#define USP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define USP_MAX_WORLD 32   /* largest P */
+#define USP_MAX_HEADS 256  /* largest H */
+
+enum usp_status {
+  USP_OK = 0,
+  USP_ERR_INVALID_ARG = 1, /* null pointer, bad count, P < 1, T < P, H < P ...   */
+  USP_ERR_SHAPE = 2,       /* sizes that do not fit the plan                      */
+  USP_ERR_DTYPE = 3,       /* unknown element type                                */
+  USP_ERR_ALIGN = 4,       /* pointer or row size not 16-byte aligned             */
+  USP_ERR_CUDA = 5,        /* a CUDA runtime call failed (message has the name)    */
+  USP_ERR_TIMEOUT = 6,     /* a device-side wait ran out (see usp_device_status)  */
+  USP_ERR_UNSUPPORTED = 7, /* valid but not built (e.g. head_dim > 256)           */
+  USP_ERR_NO_DEVICE = 8    /* no CUDA device is visible                           */
+};
+
+enum usp_dtype { USP_BF16 = 0, USP_FP32 = 1, USP_FP16 = 2 };
+
+typedef struct usp_plan usp_plan;
+
+/* Thread-local text of the last failure in this thread ("" if none). */
+const char* usp_last_error_message(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int usp_version(void);
+
+/*
+ * usp_balanced_ranges -- "h3_blackwell_runtime/distributed.py", balanced_ranges.
+ * Splits `total` ordered items into `parts` contiguous non-empty ranges; the
+ * first total % parts ranges are one longer. Writes parts starts and lengths.
+ * USP_ERR_INVALID_ARG if parts < 1, total < parts, or an output is NULL.
+ */
+int usp_balanced_ranges(int64_t total, int32_t parts, int64_t* starts, int64_t* lengths);
+
+/*
+ * usp_seq_split -- API page, sp_seq_split: per-rank token counts summing to
+ * `total`, earlier ranks taking the remainder. Writes `world` counts.
+ * USP_ERR_INVALID_ARG if world < 1 or total < world (the transport page's rule).
+ */
+int usp_seq_split(int64_t total, int32_t world, int64_t* out_counts);
+
+/*
+ * usp_head_chunk_ranges -- "maxdiffusion PR #428", ulysses_attention_chunks:
+ * local-head windows of the head-chunked passes. With s = ceil(G/num_chunks),
+ * chunk c is [c*s, min((c+1)*s, G)); empty chunks are dropped. Writes the
+ * number of chunks to *n_out and the windows to lo[]/hi[] (capacity >= G).
+ * USP_ERR_INVALID_ARG if group_heads < 1 or num_chunks < 1.
+ */
+int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_out, int32_t* lo,
+                          int32_t* hi);
+
+/*
+ * usp_plan_create -- "h3_blackwell_runtime/distributed.py",
+ * SequenceParallelContext.create: the token and head ownership of all P
+ * virtual ranks (both balanced), for tensors of B x T' x H x D elements of
+ * `dtype`, with `prefix_tokens` (0 or 1) replicated leading tokens
+ * ("deepspeed/sequence/autosp_vit.py": the cls token is replicated on every
+ * rank). Binds the plan to the current CUDA device and creates one auxiliary
+ * stream and its events there (used to overlap head chunks).
+ * Errors: USP_ERR_INVALID_ARG (world < 1 or > USP_MAX_WORLD, seq_len < world,
+ * heads < world or > USP_MAX_HEADS, batch < 1, head_dim < 1, prefix not 0/1),
+ * USP_ERR_DTYPE, USP_ERR_NO_DEVICE, USP_ERR_CUDA.
+ */
+int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads,
+                    int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens);
+
+/* Releases the plan (synchronises its auxiliary stream first). NULL is ignored. */
+int usp_plan_destroy(usp_plan* plan);
+
+/* Copies the plan's ownership tables out; any output may be NULL. Arrays hold `world` entries. */
+int usp_plan_query(const usp_plan* plan, int64_t* tok_start, int64_t* tok_len, int32_t* head_start,
+                   int32_t* head_len);
+
+/*
+ * usp_scatter_sequence -- API page, scatter_sequence: each rank's contiguous
+ * token window of a replicated tensor, materialised into that rank's buffer.
+ * x_full is [outer, T', row] and x_shards[r] is [outer, prefix + T_r, row],
+ * `row` = row_bytes bytes per token (a multiple of 16). The prefix rows are
+ * copied to every shard. outer = 0 and row_bytes = 0 mean B and H*D*elem.
+ */
+int usp_scatter_sequence(const usp_plan* plan, const void* x_full, void* const* x_shards,
+                         int64_t outer, int64_t row_bytes, void* stream);
+
+/*
+ * usp_gather_sequence -- API page, gather_sequence: the full tensor from the
+ * shards in rank order (no padding is needed between virtual ranks). Shapes
+ * as usp_scatter_sequence; the prefix rows are taken from rank 0.
+ */
+int usp_gather_sequence(const usp_plan* plan, const void* const* x_shards, void* x_full,
+                        int64_t outer, int64_t row_bytes, void* stream);
+
+/*
+ * usp_sp_head_slice -- API page, sp_head_slice: rank r keeps heads
+ * [h0_r, h0_r + H_r) of x_full [rows, H, D] into x_head_shards[r] [rows, H_r, D].
+ * These are the heads the seq->head exchange routes to rank r. rows = 0 means B*T'.
+ */
+int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards,
+                      int64_t rows, void* stream);
+
+/* usp_sp_head_gather -- API page, sp_head_gather: inverse of usp_sp_head_slice. */
+int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, void* x_full,
+                       int64_t rows, void* stream);
+
+/*
+ * usp_ulysses_seq_to_head -- "h3_blackwell_runtime/distributed.py",
+ * SequenceParallelContext.seq_to_heads: for each of `ntensors` (1..3) tensors
+ * (q, k, v), sequence shards in[t*P + i] [B, prefix+T_i, H, D] become head
+ * shards out[t*P + r] [B, T', H_r, D]:
+ *   out_r[b, prefix + t0_i + t, h, :] = in_i[b, prefix + t, h0_r + h, :]
+ * and the prefix rows of every out_r come from rank 0's shard.
+ * Outputs must not overlap inputs.
+ */
+int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* const* in,
+                            void* const* out, void* stream);
+
+/*
+ * usp_ulysses_head_to_seq -- "h3_blackwell_runtime/distributed.py",
+ * SequenceParallelContext.heads_to_seq: head shards in[t*P + r] [B, T', H_r, D]
+ * become sequence shards out[t*P + i] [B, prefix+T_i, H, D]:
+ *   out_i[b, prefix + t, h0_r + h, :] = in_r[b, prefix + t0_i + t, h, :]
+ * and every rank receives the prefix rows.
+ */
+int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* const* in,
+                            void* const* out, void* stream);
+
+/*
+ * usp_head_attention -- API page, ulysses_attention's run_attention: the
+ * unchanged single-device attention on every rank's head shard,
+ *   o_r[b, :, h, :] = softmax(q_r[b, :, h, :] k_r[b, :, h, :]^T * scale) v_r[b, :, h, :]
+ * non-causal, no mask, over all T' tokens ("deepspeed/sequence/autosp_vit.py":
+ * ViT attention is non-causal). scale <= 0 selects 1/sqrt(D). 16-bit types
+ * accumulate in fp32 on the tensor cores (tcgen05) with P rounded to the
+ * input type; fp32 runs in fp32 on the CUDA cores.
+ */
+int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const void* const* k_heads,
+                       const void* const* v_heads, void* const* o_heads, float scale, void* stream);
+
+/*
+ * usp_ulysses_attention_workspace_size -- bytes of device workspace that
+ * usp_ulysses_attention needs (the head-sharded q, k and v of all ranks).
+ */
+int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunks, size_t* bytes);
+
+/*
+ * usp_ulysses_attention -- API page, ulysses_attention, with the head-chunked
+ * passes of "maxdiffusion PR #428": sequence shards q/k/v[i]
+ * [B, prefix+T_i, H, D] in, sequence shards out[i] [B, prefix+T_i, H, D] out.
+ * For each head chunk c (usp_head_chunk_ranges over G = max H_r, the same
+ * local-head window on every rank, clipped to H_r): the seq->head exchange of
+ * chunk c's heads of q, k and v runs on the plan's auxiliary stream; the
+ * attention of chunk c runs on `stream` once that exchange is done, and its
+ * epilogue writes every output row straight to the sequence shard of the rank
+ * that owns the row's token (the head->seq exchange, fused). The exchange of
+ * chunk c+1 overlaps the attention of chunk c. The result does not depend on
+ * num_chunks beyond rounding-free identity: heads are independent.
+ * workspace: caller-owned device memory of at least
+ * usp_ulysses_attention_workspace_size() bytes, 256-byte aligned; its
+ * contents are scratch. Outputs must not overlap inputs or the workspace.
+ */
+int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void* const* k,
+                          const void* const* v, void* const* out, float scale, int32_t num_chunks,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * usp_device_status -- synchronises the current device, then reads the
+ * library's device-side error word of its kernels (0 = no error; nonzero =
+ * a bounded device-side wait ran out, and identifies the wait). reset != 0
+ * clears it. Diagnostic only.
+ */
+int usp_device_status(uint32_t* code, int32_t reset);
+
+/*
+ * usp_debug_wait_timeout -- launches one CTA that waits on a barrier nothing
+ * arrives on, with a limit of `limit_us` microseconds (1..2000000); the wait
+ * gives up, records the error word and returns. Used to test that a wait that
+ * runs out reports USP_ERR_TIMEOUT through usp_device_status without faulting
+ * or hanging the GPU.
+ */
+int usp_debug_wait_timeout(uint32_t limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* USP_H_ */

@@ -1,0 +1,146 @@
+// Non-causal softmax attention in fp32 on the CUDA cores.
+//
+// Same operation and output routing as the tcgen05 kernel (API page
+// "mstar.model.components.distributed.sequence_parallel", ulysses_attention /
+// run_attention), for fp32 inputs, where the tensor-core fp32 paths (tf32)
+// would not hold fp32 accuracy. Four threads share one query row; each holds a
+// quarter of the head dimension of q and of the accumulator. Keys and values
+// are staged through shared memory 32 rows at a time; the online softmax runs
+// in the log2 domain with exact exp2f.
+#include <cmath>
+
+#include "device_common.cuh"
+#include "usp_internal.h"
+
+namespace usp {
+namespace {
+
+constexpr int kTPR = 4;                  // threads per query row
+constexpr int kThreads = 128;
+constexpr int kRows = kThreads / kTPR;   // query rows per CTA
+constexpr int kKT = 32;                  // keys per smem tile
+
+template <int DPT>
+__global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_constant__ AttnLaunch L, float scale_log2) {
+  extern __shared__ float sh[];
+  const int D = L.head_dim;
+  const int DP = DPT * kTPR;  // padded head dim
+  float* sk = sh;
+  float* sv = sh + kKT * DP;
+
+  const int hi = blockIdx.y / L.batch;
+  const int b = blockIdx.y - hi * L.batch;
+  const int hm = L.heads[hi];
+  const int T = L.tokens;
+  const int sub = threadIdx.x % kTPR;
+  const int row = blockIdx.x * kRows + threadIdx.x / kTPR;
+  const bool row_ok = row < T;
+
+  const float* qb = static_cast<const float*>(L.in.q) + hm * L.in.stride_head + b * L.in.stride_batch;
+  const float* kb = static_cast<const float*>(L.in.k) + hm * L.in.stride_head + b * L.in.stride_batch;
+  const float* vb = static_cast<const float*>(L.in.v) + hm * L.in.stride_head + b * L.in.stride_batch;
+
+  float q[DPT], acc[DPT];
+#pragma unroll
+  for (int i = 0; i < DPT; ++i) {
+    const int d = sub * DPT + i;
+    q[i] = (row_ok && d < D) ? qb[static_cast<int64_t>(row) * L.in.stride_token + d] * scale_log2 : 0.f;
+    acc[i] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+
+  for (int k0 = 0; k0 < T; k0 += kKT) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kKT * DP; idx += kThreads) {
+      const int r = idx / DP, d = idx - r * DP;
+      const bool ok = (k0 + r < T) && d < D;
+      const int64_t off = static_cast<int64_t>(k0 + r) * L.in.stride_token + d;
+      sk[idx] = ok ? kb[off] : 0.f;
+      sv[idx] = ok ? vb[off] : 0.f;
+    }
+    __syncthreads();
+    const int nk = min(kKT, T - k0);
+    float s[kKT];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kKT; ++r) {
+      float dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) dot = fmaf(q[i], sk[r * DP + sub * DPT + i], dot);
+#pragma unroll
+      for (int o = 1; o < kTPR; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      s[r] = (r < nk) ? dot : -INFINITY;
+      mx = fmaxf(mx, s[r]);
+    }
+    const float m_new = fmaxf(m, mx);
+    const float alpha = exp2f(m - m_new);
+    l *= alpha;
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int r = 0; r < kKT; ++r) {
+      const float pr = exp2f(s[r] - m_new);
+      l += pr;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) acc[i] = fmaf(pr, sv[r * DP + sub * DPT + i], acc[i]);
+    }
+    m = m_new;
+  }
+  if (!row_ok) return;
+
+  const AttnOut& out = L.out;
+  int seg_lo, seg_hi;
+  int64_t row_in_seg;
+  if (row < out.prefix) {
+    seg_lo = 0;
+    seg_hi = out.nseg;
+    row_in_seg = row;
+  } else {
+    const int64_t tok = row - out.prefix;
+    int s = 0;
+    while (s + 1 < out.nseg && tok >= out.seg_start[s + 1]) ++s;
+    seg_lo = s;
+    seg_hi = s + 1;
+    row_in_seg = out.prefix + tok - out.seg_start[s];
+  }
+  const float inv_l = 1.f / l;
+  for (int s = seg_lo; s < seg_hi; ++s) {
+    const int64_t rows_s = out.prefix + out.seg_len[s];
+    float* dst = static_cast<float*>(out.seg_ptr[s]) + ((b * rows_s + row_in_seg) * out.out_heads + hm) * D;
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) {
+      const int d = sub * DPT + i;
+      if (d < D) dst[d] = acc[i] * inv_l;
+    }
+  }
+}
+
+template <int DPT>
+int launch_dpt(const AttnLaunch& L, cudaStream_t stream) {
+  const size_t smem = 2 * kKT * DPT * kTPR * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<DPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(simt smem)");
+  }
+  const float scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
+  dim3 grid((L.tokens + kRows - 1) / kRows, L.batch * L.n_heads);
+  attn_simt_kernel<DPT><<<grid, kThreads, smem, stream>>>(L, scale_log2);
+  return cuda_check(cudaGetLastError(), "attention (fp32) launch");
+}
+
+}  // namespace
+
+int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream) {
+  if (L.n_heads == 0 || L.batch == 0 || L.tokens == 0) return USP_OK;
+  if (L.dtype != USP_FP32) return set_error(USP_ERR_UNSUPPORTED, "fp32 attention kernel called with a 16-bit type");
+  const int D = L.head_dim;
+  if (D <= 16) return launch_dpt<4>(L, stream);
+  if (D <= 32) return launch_dpt<8>(L, stream);
+  if (D <= 64) return launch_dpt<16>(L, stream);
+  if (D <= 128) return launch_dpt<32>(L, stream);
+  if (D <= 256) return launch_dpt<64>(L, stream);
+  return set_error(USP_ERR_UNSUPPORTED, "head_dim %d > 256 is not built", D);
+}
+
+}  // namespace usp

@@ -1,0 +1,131 @@
+// Ragged row permutation between sequence shards and head shards.
+//
+// Every layout step of the Ulysses block moves whole head units (D elements)
+// between a buffer that holds complete token rows (the "sequence side") and a
+// buffer that holds a contiguous head range for every token (the "head
+// side"):
+//   seq->head exchange  ("h3_blackwell_runtime/distributed.py", seq_to_heads)
+//   head->seq exchange  (heads_to_seq)
+//   scatter / gather of the sequence, head slice / gather (API page)
+// The kernel walks the sequence-side rows, so that side is read or written in
+// full contiguous rows; each head unit is a contiguous run of D*elem bytes on
+// the head side. One warp moves one row at a time with vector loads of
+// 2..16 bytes, all loads of a batch issued before their stores.
+#include <cstdio>
+
+#include "device_common.cuh"
+#include "usp_internal.h"
+
+namespace usp {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+template <typename V>
+__global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant__ PermuteArgs a) {
+  __shared__ int32_t s_unit[USP_MAX_HEADS];    // head unit index on the sequence side
+  __shared__ int32_t s_rank[USP_MAX_HEADS];    // head-side buffer
+  __shared__ int32_t s_local[USP_MAX_HEADS];   // unit index inside that buffer
+  __shared__ int32_t s_count[USP_MAX_HEADS];   // units held by that buffer
+  for (int i = threadIdx.x; i < a.nsel; i += blockDim.x) {
+    const int h = a.sel_head[i];
+    const int r = a.sel_rank[i];
+    s_unit[i] = h;
+    s_rank[i] = r;
+    s_local[i] = h - a.head_start[r];
+    s_count[i] = a.head_start[r + 1] - a.head_start[r];
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  const int64_t total_rows = a.seq_rows[a.n_seq];
+  const int nvec = a.nsel * a.dv;
+
+  for (int64_t row = warp; row < total_rows; row += nwarps) {
+    int s = 0;
+    while (a.seq_rows[s + 1] <= row) ++s;
+    const int64_t rr = row - a.seq_rows[s];
+    const int64_t rows_per_b = a.prefix + a.tok_len[s];
+    const int64_t b = rr / rows_per_b;
+    const int64_t tl = rr - b * rows_per_b;
+    // Replicated prefix rows: read once (from buffer 0) on the way to the head
+    // side, written to every sequence-side buffer on the way back.
+    if (a.dir == 0 && tl < a.prefix && s != 0) continue;
+    const int64_t t = (tl < a.prefix) ? tl : a.prefix + a.tok_start[s] + (tl - a.prefix);
+    const int64_t seq_base = rr * a.heads * a.dv;
+
+    for (int j0 = 0; j0 < nvec; j0 += 32 * kUnroll) {
+      int64_t soff[kUnroll], hoff[kUnroll];
+      int hr[kUnroll];
+      bool ok[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = j0 + u * 32 + lane;
+        ok[u] = j < nvec;
+        const int k = ok[u] ? j / a.dv : 0;
+        const int d = j - k * a.dv;
+        const int64_t hl = s_local[k];
+        const int64_t cr = s_count[k];
+        hr[u] = s_rank[k];
+        soff[u] = seq_base + static_cast<int64_t>(s_unit[k]) * a.dv + d;
+        hoff[u] = (a.head_layout == 0) ? ((b * a.full_tokens + t) * cr + hl) * a.dv + d
+                                       : ((hl * a.outer + b) * a.full_tokens + t) * a.dv + d;
+      }
+      for (int ti = 0; ti < a.ntensors; ++ti) {
+        V val[kUnroll];
+        if (a.dir == 0) {
+          const V* src = static_cast<const V*>(a.seq_ptr[ti][s]);
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (ok[u]) val[u] = __ldcs(src + soff[u]);
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (ok[u]) __stcs(static_cast<V*>(a.head_ptr[ti][hr[u]]) + hoff[u], val[u]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (ok[u]) val[u] = __ldcs(static_cast<const V*>(a.head_ptr[ti][hr[u]]) + hoff[u]);
+          V* dst = static_cast<V*>(a.seq_ptr[ti][s]);
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (ok[u]) __stcs(dst + soff[u], val[u]);
+        }
+      }
+    }
+  }
+}
+
+int sm_count() {
+  static int count = 0;
+  if (count == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      count = 148;
+  }
+  return count;
+}
+
+}  // namespace
+
+int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream) {
+  const int64_t rows = a.seq_rows[a.n_seq];
+  if (rows == 0 || a.nsel == 0) return USP_OK;
+  const int64_t warps_needed = rows;
+  int64_t blocks = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 resident CTAs of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  dim3 grid(static_cast<unsigned>(blocks)), block(kThreads);
+  switch (vec_bytes) {
+    case 16: permute_kernel<uint4><<<grid, block, 0, stream>>>(a); break;
+    case 8: permute_kernel<uint2><<<grid, block, 0, stream>>>(a); break;
+    case 4: permute_kernel<uint32_t><<<grid, block, 0, stream>>>(a); break;
+    case 2: permute_kernel<uint16_t><<<grid, block, 0, stream>>>(a); break;
+    default: return set_error(USP_ERR_INVALID_ARG, "internal: bad vector width %d", vec_bytes);
+  }
+  return cuda_check(cudaGetLastError(), "permute kernel launch");
+}
+
+}  // namespace usp

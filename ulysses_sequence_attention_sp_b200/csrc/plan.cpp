@@ -1,0 +1,577 @@
+// C ABI of libusp: plan (ragged token/head ownership of P virtual ranks),
+// argument checking, and the launch sequence of every entry point.
+//
+// Ownership and splits follow "h3_blackwell_runtime/distributed.py -- Ragged
+// Ulysses sequence-parallel transport" (balanced_ranges,
+// SequenceParallelContext); the entry points follow the API page
+// "mstar.model.components.distributed.sequence_parallel"; head chunks follow
+// "maxdiffusion PR #428: experimental two-phase (head-chunked) Ulysses
+// all-to-all"; the replicated cls prefix follows "deepspeed/sequence/autosp_vit.py".
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "usp_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(int dtype) {
+  switch (dtype) {
+    case USP_BF16:
+    case USP_FP16: return 2;
+    case USP_FP32: return 4;
+    default: return 0;
+  }
+}
+
+// Balanced contiguous non-empty split: the first total % parts ranges take one more.
+int balanced(int64_t total, int32_t parts, int64_t* starts, int64_t* lengths) {
+  if (parts < 1) return usp::set_error(USP_ERR_INVALID_ARG, "parts must be positive (got %d)", parts);
+  if (total < parts)
+    return usp::set_error(USP_ERR_INVALID_ARG, "cannot split %lld items into %d non-empty ranges",
+                          static_cast<long long>(total), parts);
+  const int64_t base = total / parts, extra = total % parts;
+  int64_t start = 0;
+  for (int32_t r = 0; r < parts; ++r) {
+    const int64_t len = base + (r < extra ? 1 : 0);
+    if (starts) starts[r] = start;
+    if (lengths) lengths[r] = len;
+    start += len;
+  }
+  return USP_OK;
+}
+
+int check_plan(const usp_plan* plan) {
+  if (!plan) return usp::set_error(USP_ERR_INVALID_ARG, "plan is NULL");
+  return USP_OK;
+}
+
+int check_ptrs(const void* const* ptrs, int n, const char* what) {
+  if (!ptrs) return usp::set_error(USP_ERR_INVALID_ARG, "%s: pointer array is NULL", what);
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) return usp::set_error(USP_ERR_INVALID_ARG, "%s[%d] is NULL", what, i);
+    if (!aligned16(ptrs[i])) return usp::set_error(USP_ERR_ALIGN, "%s[%d] is not 16-byte aligned", what, i);
+  }
+  return USP_OK;
+}
+
+int check_ptr(const void* p, const char* what) {
+  if (!p) return usp::set_error(USP_ERR_INVALID_ARG, "%s is NULL", what);
+  if (!aligned16(p)) return usp::set_error(USP_ERR_ALIGN, "%s is not 16-byte aligned", what);
+  return USP_OK;
+}
+
+// Largest vector width (16/8/4/2 bytes) dividing the head-unit size.
+int pick_vec(int64_t unit_bytes) {
+  for (int v : {16, 8, 4, 2})
+    if (unit_bytes % v == 0) return v;
+  return 0;
+}
+
+int device_matches(const usp_plan* plan) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return usp::cuda_check(e, "cudaGetDevice");
+  if (dev != plan->device)
+    return usp::set_error(USP_ERR_INVALID_ARG, "plan was created on device %d but device %d is current", plan->device,
+                          dev);
+  return USP_OK;
+}
+
+// Fills the parts of PermuteArgs that describe the plan's ranks.
+void fill_seq_side(usp::PermuteArgs& a, const usp_plan* p, int64_t outer) {
+  a.n_seq = p->world;
+  a.prefix = p->prefix;
+  a.outer = outer;
+  a.seq_rows[0] = 0;
+  for (int s = 0; s < p->world; ++s) {
+    a.tok_start[s] = p->tok_start[s];
+    a.tok_len[s] = p->tok_len[s];
+    a.seq_rows[s + 1] = a.seq_rows[s] + outer * (p->prefix + p->tok_len[s]);
+  }
+}
+
+void select_all_heads(usp::PermuteArgs& a, int heads, const int32_t* head_start, int nranks) {
+  a.nsel = heads;
+  int r = 0;
+  for (int h = 0; h < heads; ++h) {
+    while (r + 1 < nranks && h >= head_start[r + 1]) ++r;
+    a.sel_head[h] = static_cast<uint16_t>(h);
+    a.sel_rank[h] = static_cast<uint8_t>(r);
+  }
+}
+
+// Heads of local window [lo, hi) on every rank (ragged: clipped to H_r).
+void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) {
+  a.nsel = 0;
+  for (int r = 0; r < p->world; ++r)
+    for (int h = lo; h < hi && h < p->head_len[r]; ++h) {
+      a.sel_head[a.nsel] = static_cast<uint16_t>(p->head_start[r] + h);
+      a.sel_rank[a.nsel] = static_cast<uint8_t>(r);
+      ++a.nsel;
+    }
+}
+
+int seq_head_exchange(const usp_plan* plan, int dir, int32_t ntensors, const void* const* seq, void* const* heads,
+                      cudaStream_t stream) {
+  usp::PermuteArgs a;
+  memset(&a, 0, sizeof(a));
+  const int64_t unit = static_cast<int64_t>(plan->head_dim) * plan->elem;
+  const int vec = pick_vec(unit);
+  a.dir = dir;
+  fill_seq_side(a, plan, plan->batch);
+  a.n_head = plan->world;
+  a.ntensors = ntensors;
+  a.heads = plan->heads;
+  a.dv = static_cast<int32_t>(unit / vec);
+  a.head_layout = 0;
+  a.full_tokens = plan->tokens();
+  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = plan->head_start[r];
+  select_all_heads(a, plan->heads, plan->head_start, plan->world);
+  for (int t = 0; t < ntensors; ++t)
+    for (int r = 0; r < plan->world; ++r) {
+      a.seq_ptr[t][r] = const_cast<void*>(seq[t * plan->world + r]);
+      a.head_ptr[t][r] = heads[t * plan->world + r];
+    }
+  return usp::launch_permute(a, vec, stream);
+}
+
+}  // namespace
+
+namespace usp {
+
+int set_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return USP_OK;
+  return set_error(USP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+}  // namespace usp
+
+extern "C" {
+
+const char* usp_last_error_message(void) { return g_last_error.c_str(); }
+
+int usp_version(void) { return 100; }
+
+int usp_balanced_ranges(int64_t total, int32_t parts, int64_t* starts, int64_t* lengths) {
+  if (!starts || !lengths) return usp::set_error(USP_ERR_INVALID_ARG, "output arrays must not be NULL");
+  return balanced(total, parts, starts, lengths);
+}
+
+int usp_seq_split(int64_t total, int32_t world, int64_t* out_counts) {
+  if (!out_counts) return usp::set_error(USP_ERR_INVALID_ARG, "out_counts is NULL");
+  return balanced(total, world, nullptr, out_counts);
+}
+
+int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_out, int32_t* lo, int32_t* hi) {
+  if (!n_out || !lo || !hi) return usp::set_error(USP_ERR_INVALID_ARG, "output pointers must not be NULL");
+  if (group_heads < 1) return usp::set_error(USP_ERR_INVALID_ARG, "group_heads must be positive");
+  if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive");
+  const int32_t size = (group_heads + num_chunks - 1) / num_chunks;
+  int32_t n = 0;
+  for (int32_t a = 0; a < group_heads; a += size, ++n) {
+    lo[n] = a;
+    hi[n] = a + size < group_heads ? a + size : group_heads;
+  }
+  *n_out = n;
+  return USP_OK;
+}
+
+int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim, int32_t world,
+                    int32_t dtype, int32_t prefix_tokens) {
+  if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (world < 1 || world > USP_MAX_WORLD)
+    return usp::set_error(USP_ERR_INVALID_ARG, "world must be in [1, %d] (got %d)", USP_MAX_WORLD, world);
+  if (batch < 1) return usp::set_error(USP_ERR_INVALID_ARG, "batch must be positive");
+  if (head_dim < 1) return usp::set_error(USP_ERR_INVALID_ARG, "head_dim must be positive");
+  if (heads > USP_MAX_HEADS) return usp::set_error(USP_ERR_INVALID_ARG, "heads must be <= %d", USP_MAX_HEADS);
+  if (prefix_tokens != 0 && prefix_tokens != 1)
+    return usp::set_error(USP_ERR_INVALID_ARG, "prefix_tokens must be 0 or 1 (got %d)", prefix_tokens);
+  const int e = elem_bytes(dtype);
+  if (!e) return usp::set_error(USP_ERR_DTYPE, "unknown dtype %d", dtype);
+  usp_plan* p = new usp_plan();
+  p->batch = batch;
+  p->seq_len = seq_len;
+  p->heads = heads;
+  p->head_dim = head_dim;
+  p->world = world;
+  p->dtype = dtype;
+  p->prefix = prefix_tokens;
+  p->elem = e;
+  int rc = balanced(seq_len, world, p->tok_start, p->tok_len);
+  if (rc == USP_OK) {
+    int64_t hs[USP_MAX_WORLD], hl[USP_MAX_WORLD];
+    rc = balanced(heads, world, hs, hl);
+    if (rc == USP_OK) {
+      for (int r = 0; r < world; ++r) {
+        p->head_start[r] = static_cast<int32_t>(hs[r]);
+        p->head_len[r] = static_cast<int32_t>(hl[r]);
+      }
+      p->head_start[world] = heads;
+      p->group_heads = p->head_len[0];
+    }
+  }
+  if (rc != USP_OK) {
+    delete p;
+    return rc;
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    delete p;
+    return usp::set_error(USP_ERR_NO_DEVICE, "no CUDA device is visible");
+  }
+  cudaError_t ce = cudaGetDevice(&p->device);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&p->aux, cudaStreamNonBlocking);
+  if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&p->ev_inputs, cudaEventDisableTiming);
+  for (int c = 0; ce == cudaSuccess && c < p->group_heads; ++c) {
+    cudaEvent_t ev;
+    ce = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (ce == cudaSuccess) p->ev_chunk.push_back(ev);
+  }
+  if (ce != cudaSuccess) {
+    rc = usp::cuda_check(ce, "plan stream/event creation");
+    usp_plan_destroy(p);
+    return rc;
+  }
+  *out = p;
+  return USP_OK;
+}
+
+int usp_plan_destroy(usp_plan* plan) {
+  if (!plan) return USP_OK;
+  if (plan->aux) {
+    cudaStreamSynchronize(plan->aux);
+    cudaStreamDestroy(plan->aux);
+  }
+  if (plan->ev_inputs) cudaEventDestroy(plan->ev_inputs);
+  for (cudaEvent_t ev : plan->ev_chunk) cudaEventDestroy(ev);
+  delete plan;
+  return USP_OK;
+}
+
+int usp_plan_query(const usp_plan* plan, int64_t* tok_start, int64_t* tok_len, int32_t* head_start,
+                   int32_t* head_len) {
+  if (int rc = check_plan(plan)) return rc;
+  for (int r = 0; r < plan->world; ++r) {
+    if (tok_start) tok_start[r] = plan->tok_start[r];
+    if (tok_len) tok_len[r] = plan->tok_len[r];
+    if (head_start) head_start[r] = plan->head_start[r];
+    if (head_len) head_len[r] = plan->head_len[r];
+  }
+  return USP_OK;
+}
+
+// scatter: the full tensor is the head side with a single head unit per row.
+static int scatter_gather(const usp_plan* plan, int dir, const void* full, void* const* shards, int64_t outer,
+                          int64_t row_bytes, cudaStream_t stream) {
+  if (outer == 0) outer = plan->batch;
+  if (row_bytes == 0) row_bytes = static_cast<int64_t>(plan->heads) * plan->head_dim * plan->elem;
+  if (outer < 1 || row_bytes < 1) return usp::set_error(USP_ERR_SHAPE, "outer and row_bytes must be positive");
+  if (row_bytes % 16 != 0) return usp::set_error(USP_ERR_ALIGN, "row_bytes must be a multiple of 16");
+  usp::PermuteArgs a;
+  memset(&a, 0, sizeof(a));
+  a.dir = dir;
+  fill_seq_side(a, plan, outer);
+  a.n_head = 1;
+  a.ntensors = 1;
+  a.heads = 1;
+  a.dv = static_cast<int32_t>(row_bytes / 16);
+  a.head_layout = 0;
+  a.full_tokens = plan->tokens();
+  a.head_start[0] = 0;
+  a.head_start[1] = 1;
+  a.nsel = 1;
+  a.sel_head[0] = 0;
+  a.sel_rank[0] = 0;
+  a.head_ptr[0][0] = const_cast<void*>(full);
+  for (int r = 0; r < plan->world; ++r) a.seq_ptr[0][r] = shards[r];
+  return usp::launch_permute(a, 16, stream);
+}
+
+int usp_scatter_sequence(const usp_plan* plan, const void* x_full, void* const* x_shards, int64_t outer,
+                         int64_t row_bytes, void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptr(x_full, "x_full")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(x_shards), plan->world, "x_shards")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return scatter_gather(plan, 1, x_full, x_shards, outer, row_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int usp_gather_sequence(const usp_plan* plan, const void* const* x_shards, void* x_full, int64_t outer,
+                        int64_t row_bytes, void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptr(x_full, "x_full")) return rc;
+  if (int rc = check_ptrs(x_shards, plan->world, "x_shards")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return scatter_gather(plan, 0, x_full, const_cast<void* const*>(x_shards), outer, row_bytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
+// head slice: the full tensor is a single sequence-side buffer of `rows` rows.
+static int head_slice_gather(const usp_plan* plan, int dir, const void* full, void* const* shards, int64_t rows,
+                             cudaStream_t stream) {
+  if (rows == 0) rows = plan->batch * plan->tokens();
+  if (rows < 1) return usp::set_error(USP_ERR_SHAPE, "rows must be positive");
+  const int64_t unit = static_cast<int64_t>(plan->head_dim) * plan->elem;
+  const int vec = pick_vec(unit);
+  usp::PermuteArgs a;
+  memset(&a, 0, sizeof(a));
+  a.dir = dir;
+  a.n_seq = 1;
+  a.prefix = 0;
+  a.outer = 1;
+  a.seq_rows[0] = 0;
+  a.seq_rows[1] = rows;
+  a.tok_start[0] = 0;
+  a.tok_len[0] = rows;
+  a.n_head = plan->world;
+  a.ntensors = 1;
+  a.heads = plan->heads;
+  a.dv = static_cast<int32_t>(unit / vec);
+  a.head_layout = 0;
+  a.full_tokens = rows;
+  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = plan->head_start[r];
+  select_all_heads(a, plan->heads, plan->head_start, plan->world);
+  a.seq_ptr[0][0] = const_cast<void*>(full);
+  for (int r = 0; r < plan->world; ++r) a.head_ptr[0][r] = shards[r];
+  return usp::launch_permute(a, vec, stream);
+}
+
+int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards, int64_t rows,
+                      void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptr(x_full, "x_full")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(x_head_shards), plan->world, "x_head_shards")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return head_slice_gather(plan, 0, x_full, x_head_shards, rows, static_cast<cudaStream_t>(stream));
+}
+
+int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, void* x_full, int64_t rows,
+                       void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptr(x_full, "x_full")) return rc;
+  if (int rc = check_ptrs(x_head_shards, plan->world, "x_head_shards")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return head_slice_gather(plan, 1, x_full, const_cast<void* const*>(x_head_shards), rows,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
+                            void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
+  if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return seq_head_exchange(plan, 0, ntensors, in, out, static_cast<cudaStream_t>(stream));
+}
+
+int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
+                            void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
+  if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return seq_head_exchange(plan, 1, ntensors, const_cast<const void* const*>(out), const_cast<void* const*>(in),
+                           static_cast<cudaStream_t>(stream));
+}
+
+static int check_attention_shape(const usp_plan* plan) {
+  if (plan->tokens() > (int64_t(1) << 30)) return usp::set_error(USP_ERR_SHAPE, "too many tokens");
+  if (plan->dtype == USP_FP32) {
+    if (plan->head_dim > 256) return usp::set_error(USP_ERR_UNSUPPORTED, "fp32 attention: head_dim > 256 not built");
+  } else if (!usp::attention_tc_supported(plan->dtype, plan->head_dim)) {
+    return usp::set_error(USP_ERR_UNSUPPORTED,
+                          "16-bit attention needs head_dim a multiple of 16 in [16, 128] (got %d)", plan->head_dim);
+  }
+  return USP_OK;
+}
+
+static int launch_attention(const usp::AttnLaunch& L, cudaStream_t stream) {
+  return L.dtype == USP_FP32 ? usp::launch_attention_simt(L, stream) : usp::launch_attention_tc(L, stream);
+}
+
+static float resolve_scale(const usp_plan* plan, float scale) {
+  return scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(plan->head_dim)));
+}
+
+int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const void* const* k_heads,
+                       const void* const* v_heads, void* const* o_heads, float scale, void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptrs(q_heads, plan->world, "q_heads")) return rc;
+  if (int rc = check_ptrs(k_heads, plan->world, "k_heads")) return rc;
+  if (int rc = check_ptrs(v_heads, plan->world, "v_heads")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(o_heads), plan->world, "o_heads")) return rc;
+  if (int rc = check_attention_shape(plan)) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t T = plan->tokens(), D = plan->head_dim;
+  for (int r = 0; r < plan->world; ++r) {
+    usp::AttnLaunch L;
+    memset(&L, 0, sizeof(L));
+    const int64_t hr = plan->head_len[r];
+    L.in = {q_heads[r], k_heads[r], v_heads[r], D, hr * D, T * hr * D, hr};
+    L.out.nseg = 1;
+    L.out.prefix = 0;
+    L.out.out_heads = static_cast<int32_t>(hr);
+    L.out.seg_start[0] = 0;
+    L.out.seg_len[0] = T;
+    L.out.seg_ptr[0] = o_heads[r];
+    L.tokens = static_cast<int32_t>(T);
+    L.batch = static_cast<int32_t>(plan->batch);
+    L.n_heads = static_cast<int32_t>(hr);
+    L.head_dim = static_cast<int32_t>(D);
+    L.dtype = plan->dtype;
+    L.scale = resolve_scale(plan, scale);
+    for (int h = 0; h < hr; ++h) L.heads[h] = static_cast<uint16_t>(h);
+    if (int rc = launch_attention(L, s)) return rc;
+  }
+  return USP_OK;
+}
+
+static size_t workspace_tensor_bytes(const usp_plan* plan) {
+  const size_t bytes = static_cast<size_t>(plan->batch) * plan->tokens() * plan->heads * plan->head_dim * plan->elem;
+  return (bytes + 255) & ~size_t(255);
+}
+
+int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunks, size_t* bytes) {
+  if (int rc = check_plan(plan)) return rc;
+  if (!bytes) return usp::set_error(USP_ERR_INVALID_ARG, "bytes is NULL");
+  if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive");
+  *bytes = 3 * workspace_tensor_bytes(plan);
+  return USP_OK;
+}
+
+int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void* const* k, const void* const* v,
+                          void* const* out, float scale, int32_t num_chunks, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive (got %d)", num_chunks);
+  if (int rc = check_ptrs(q, plan->world, "q")) return rc;
+  if (int rc = check_ptrs(k, plan->world, "k")) return rc;
+  if (int rc = check_ptrs(v, plan->world, "v")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(out), plan->world, "out")) return rc;
+  if (!workspace) return usp::set_error(USP_ERR_INVALID_ARG, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return usp::set_error(USP_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const size_t per = workspace_tensor_bytes(plan);
+  if (workspace_bytes < 3 * per)
+    return usp::set_error(USP_ERR_SHAPE, "workspace too small: %zu < %zu bytes", workspace_bytes, 3 * per);
+  if (int rc = check_attention_shape(plan)) return rc;
+  if (int rc = device_matches(plan)) return rc;
+
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t T = plan->tokens(), D = plan->head_dim, B = plan->batch, H = plan->heads;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* wq = ws;
+  void* wk = ws + per;
+  void* wv = ws + 2 * per;
+
+  // Head-chunk windows over the largest per-rank head group (rank 0's).
+  int32_t nchunks = 0;
+  int32_t lo[USP_MAX_HEADS], hi[USP_MAX_HEADS];
+  usp_head_chunk_ranges(plan->group_heads, num_chunks, &nchunks, lo, hi);
+
+  // The seq->head exchange writes a head-major workspace [H][B][T'][D]: rank r's
+  // head shard is the contiguous block of its heads, so one 4-D view of the
+  // workspace covers every rank for the attention kernel.
+  usp::PermuteArgs a;
+  memset(&a, 0, sizeof(a));
+  const int64_t unit = D * plan->elem;
+  const int vec = pick_vec(unit);
+  a.dir = 0;
+  fill_seq_side(a, plan, B);
+  a.n_head = plan->world;
+  a.ntensors = 3;
+  a.heads = static_cast<int32_t>(H);
+  a.dv = static_cast<int32_t>(unit / vec);
+  a.head_layout = 1;
+  a.full_tokens = T;
+  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = plan->head_start[r];
+  const void* src[3] = {nullptr, nullptr, nullptr};
+  void* dst[3] = {wq, wk, wv};
+  for (int r = 0; r < plan->world; ++r) {
+    a.seq_ptr[0][r] = const_cast<void*>(q[r]);
+    a.seq_ptr[1][r] = const_cast<void*>(k[r]);
+    a.seq_ptr[2][r] = const_cast<void*>(v[r]);
+    const size_t off = static_cast<size_t>(plan->head_start[r]) * B * T * D * plan->elem;
+    for (int t = 0; t < 3; ++t) a.head_ptr[t][r] = static_cast<uint8_t*>(dst[t]) + off;
+  }
+  (void)src;
+
+  usp::AttnLaunch L;
+  memset(&L, 0, sizeof(L));
+  L.in = {wq, wk, wv, B * T * D, D, T * D, H};
+  L.out.nseg = plan->world;
+  L.out.prefix = plan->prefix;
+  L.out.out_heads = static_cast<int32_t>(H);
+  for (int r = 0; r < plan->world; ++r) {
+    L.out.seg_start[r] = plan->tok_start[r];
+    L.out.seg_len[r] = plan->tok_len[r];
+    L.out.seg_ptr[r] = out[r];
+  }
+  L.tokens = static_cast<int32_t>(T);
+  L.batch = static_cast<int32_t>(B);
+  L.head_dim = static_cast<int32_t>(D);
+  L.dtype = plan->dtype;
+  L.scale = resolve_scale(plan, scale);
+
+  const bool overlap = nchunks > 1;
+  if (overlap) {
+    // Fork: the auxiliary stream packs chunk c+1 while `stream` attends chunk c.
+    if (int rc = usp::cuda_check(cudaEventRecord(plan->ev_inputs, s), "cudaEventRecord")) return rc;
+    if (int rc = usp::cuda_check(cudaStreamWaitEvent(plan->aux, plan->ev_inputs, 0), "cudaStreamWaitEvent")) return rc;
+  }
+  for (int c = 0; c < nchunks; ++c) {
+    select_chunk_heads(a, plan, lo[c], hi[c]);
+    if (overlap) {
+      if (int rc = usp::launch_permute(a, vec, plan->aux)) return rc;
+      if (int rc = usp::cuda_check(cudaEventRecord(plan->ev_chunk[c], plan->aux), "cudaEventRecord")) return rc;
+      if (int rc = usp::cuda_check(cudaStreamWaitEvent(s, plan->ev_chunk[c], 0), "cudaStreamWaitEvent")) return rc;
+    } else {
+      if (int rc = usp::launch_permute(a, vec, s)) return rc;
+    }
+    L.n_heads = a.nsel;
+    for (int i = 0; i < a.nsel; ++i) L.heads[i] = a.sel_head[i];
+    if (int rc = launch_attention(L, s)) return rc;
+  }
+  return USP_OK;
+}
+
+int usp_device_status(uint32_t* code, int32_t reset) {
+  if (!code) return usp::set_error(USP_ERR_INVALID_ARG, "code is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return usp::cuda_check(e, "cudaDeviceSynchronize");
+  if (int rc = usp::read_attention_error(code, reset != 0)) return rc;
+  if (*code != 0) {
+    usp::set_error(USP_ERR_TIMEOUT, "a device-side wait ran out (site %u)", *code);
+    return USP_ERR_TIMEOUT;
+  }
+  return USP_OK;
+}
+
+int usp_debug_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 2000000) return usp::set_error(USP_ERR_INVALID_ARG, "limit_us must be in [1, 2e6]");
+  return usp::launch_wait_timeout_probe(limit_us, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

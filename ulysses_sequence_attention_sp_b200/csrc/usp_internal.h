@@ -1,0 +1,114 @@
+// Host-side internals shared by the C ABI (plan.cpp) and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "usp.h"
+
+struct usp_plan {
+  int64_t batch = 0;
+  int64_t seq_len = 0;  // T, tokens split across ranks
+  int32_t heads = 0;
+  int32_t head_dim = 0;
+  int32_t world = 0;
+  int32_t dtype = 0;
+  int32_t prefix = 0;   // replicated leading tokens
+  int32_t elem = 0;     // bytes per element
+  int64_t tok_start[USP_MAX_WORLD] = {};
+  int64_t tok_len[USP_MAX_WORLD] = {};
+  int32_t head_start[USP_MAX_WORLD + 1] = {};
+  int32_t head_len[USP_MAX_WORLD] = {};
+  int32_t group_heads = 0;  // largest per-rank head count (rank 0's)
+  int device = 0;
+  cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
+  cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
+  std::vector<cudaEvent_t> ev_chunk;      // aux -> caller stream: chunk c packed
+
+  int64_t tokens() const { return prefix + seq_len; }
+};
+
+namespace usp {
+
+int set_error(int code, const char* fmt, ...);
+int cuda_check(cudaError_t e, const char* what);
+
+// ------------------------------------------------------------ permutation
+// One kernel moves rows between "sequence-side" buffers (each holds whole
+// token rows of H head units) and "head-side" buffers (each holds a
+// contiguous range of head units for every token). All layout operations of
+// the block are instances of it (see plan.cpp).
+struct PermuteArgs {
+  int32_t dir;          // 0: sequence side -> head side; 1: head side -> sequence side
+  int32_t n_seq;        // sequence-side buffers
+  int32_t n_head;       // head-side buffers
+  int32_t ntensors;     // tensors moved per launch (same geometry), 1..3
+  int32_t prefix;       // replicated leading rows of every sequence-side buffer
+  int32_t heads;        // head units per sequence-side row
+  int32_t dv;           // vectors per head unit
+  int32_t head_layout;  // 0: [outer][full_tokens][C_r][dv]; 1: [C_r][outer][full_tokens][dv]
+  int32_t nsel;         // head units moved (a head chunk selects a subset)
+  int32_t pad0;
+  int64_t outer;        // batch
+  int64_t full_tokens;  // rows per batch element on the head side (prefix + T)
+  int64_t seq_rows[USP_MAX_WORLD + 1];  // prefix sums of outer * (prefix + T_s)
+  int64_t tok_start[USP_MAX_WORLD];     // token offset of sequence buffer s (prefix excluded)
+  int64_t tok_len[USP_MAX_WORLD];
+  int32_t head_start[USP_MAX_WORLD + 1];  // head-unit range of head-side buffer r
+  uint16_t sel_head[USP_MAX_HEADS];       // moved head units, ascending
+  uint8_t sel_rank[USP_MAX_HEADS];        // head-side buffer owning each moved unit
+  void* seq_ptr[3][USP_MAX_WORLD];
+  void* head_ptr[3][USP_MAX_WORLD];
+};
+
+// vec_bytes in {16, 8, 4, 2}; dv counts vectors of that size.
+int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream);
+
+// -------------------------------------------------------------- attention
+// Where output rows go. Row t of (batch b, head g): rows t < prefix go to every
+// segment; other rows go to the segment s whose token range holds t - prefix.
+// Address (elements): ptr_s + ((b * (prefix + len_s) + row_in_s) * out_heads + g) * D.
+struct AttnOut {
+  int32_t nseg;
+  int32_t prefix;
+  int32_t out_heads;
+  int32_t pad0;
+  int64_t seg_start[USP_MAX_WORLD];
+  int64_t seg_len[USP_MAX_WORLD];
+  void* seg_ptr[USP_MAX_WORLD];
+};
+
+// Inputs are 4-D views (d, head, token, batch) of q, k and v; the launch
+// processes every head coordinate in heads[0..n_heads) for every batch element.
+struct AttnInputs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t stride_head;   // elements
+  int64_t stride_token;  // elements
+  int64_t stride_batch;  // elements
+  int64_t head_extent;   // head coordinates in the view
+};
+
+struct AttnLaunch {
+  AttnInputs in;
+  AttnOut out;
+  int32_t tokens;  // T' (keys and queries per head)
+  int32_t batch;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t dtype;
+  float scale;
+  uint16_t heads[USP_MAX_HEADS];
+};
+
+bool attention_tc_supported(int dtype, int head_dim);
+int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream);
+int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream);
+int read_attention_error(uint32_t* code, bool reset);
+int launch_wait_timeout_probe(uint32_t limit_us, cudaStream_t stream);
+
+}  // namespace usp

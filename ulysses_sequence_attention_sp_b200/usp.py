@@ -1,0 +1,348 @@
+"""ctypes binding of libusp (the C ABI declared in include/usp.h).
+
+Argument marshalling only: every step of the block runs in the library's CUDA
+kernels. PyTorch provides device memory (tensors) and streams. Each virtual
+rank's tensor is a separate CUDA tensor; per-rank arguments are lists indexed
+by rank. The names follow the API page "mstar.model.components.distributed.
+sequence_parallel" (sp_seq_split, scatter_sequence, gather_sequence,
+sp_head_slice, sp_head_gather, ulysses_attention) and the ragged transport
+page (seq_to_heads / heads_to_seq, here ulysses_seq_to_head /
+ulysses_head_to_seq).
+
+Loading fails loudly (OSError) if libusp.so has not been built:
+``python -m ulysses_sequence_attention_sp_b200.build``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libusp.so"
+
+USP_OK = 0
+USP_ERR_INVALID_ARG = 1
+USP_ERR_SHAPE = 2
+USP_ERR_DTYPE = 3
+USP_ERR_ALIGN = 4
+USP_ERR_CUDA = 5
+USP_ERR_TIMEOUT = 6
+USP_ERR_UNSUPPORTED = 7
+USP_ERR_NO_DEVICE = 8
+
+USP_BF16, USP_FP32, USP_FP16 = 0, 1, 2
+MAX_WORLD = 32
+MAX_HEADS = 256
+
+_DTYPES = {torch.bfloat16: USP_BF16, torch.float32: USP_FP32, torch.float16: USP_FP16}
+_NAMES = {"bf16": USP_BF16, "fp32": USP_FP32, "fp16": USP_FP16}
+_TORCH = {USP_BF16: torch.bfloat16, USP_FP32: torch.float32, USP_FP16: torch.float16}
+
+_c_i64p = ctypes.POINTER(ctypes.c_int64)
+_c_i32p = ctypes.POINTER(ctypes.c_int32)
+_c_vpp = ctypes.POINTER(ctypes.c_void_p)
+
+# name -> (restype, argtypes)
+_SIGNATURES = {
+    "usp_last_error_message": (ctypes.c_char_p, []),
+    "usp_version": (ctypes.c_int, []),
+    "usp_balanced_ranges": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, _c_i64p, _c_i64p]),
+    "usp_seq_split": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, _c_i64p]),
+    "usp_head_chunk_ranges": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _c_i32p, _c_i32p, _c_i32p]),
+    "usp_plan_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32]),
+    "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
+    "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
+                                            ctypes.c_int64, ctypes.c_void_p]),
+    "usp_gather_sequence": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, ctypes.c_void_p, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_void_p]),
+    "usp_sp_head_slice": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
+                                         ctypes.c_void_p]),
+    "usp_sp_head_gather": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, ctypes.c_void_p, ctypes.c_int64,
+                                          ctypes.c_void_p]),
+    "usp_ulysses_seq_to_head": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, _c_vpp, _c_vpp, ctypes.c_void_p]),
+    "usp_ulysses_head_to_seq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, _c_vpp, _c_vpp, ctypes.c_void_p]),
+    "usp_head_attention": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
+                                          ctypes.c_void_p]),
+    "usp_ulysses_attention_workspace_size": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32,
+                                                            ctypes.POINTER(ctypes.c_size_t)]),
+    "usp_ulysses_attention": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
+                                             ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "usp_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
+    "usp_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
+}
+
+EXPORTED = tuple(_SIGNATURES)
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _load():
+    path = library_path()
+    if not os.path.exists(path):
+        raise OSError(f"{path} is missing: build it with `python -m ulysses_sequence_attention_sp_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class UspError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"[usp error {code}] {message}")
+        self.code = code
+
+
+def _check(rc: int) -> None:
+    if rc != USP_OK:
+        raise UspError(rc, _lib.usp_last_error_message().decode())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptrs(tensors) -> ctypes.Array:
+    return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def version() -> int:
+    return _lib.usp_version()
+
+
+# ------------------------------------------------------------- partition
+def balanced_ranges(total: int, parts: int) -> tuple[tuple[int, int], ...]:
+    n = max(int(parts), 1)
+    starts, lengths = (ctypes.c_int64 * n)(), (ctypes.c_int64 * n)()
+    _check(_lib.usp_balanced_ranges(total, parts, starts, lengths))
+    return tuple((starts[i], starts[i] + lengths[i]) for i in range(parts))
+
+
+def sp_seq_split(total: int, world_size: int) -> list[int]:
+    n = max(int(world_size), 1)
+    counts = (ctypes.c_int64 * n)()
+    _check(_lib.usp_seq_split(total, world_size, counts))
+    return [counts[i] for i in range(world_size)]
+
+
+def head_chunk_ranges(group_heads: int, num_chunks: int) -> list[tuple[int, int]]:
+    cap = max(int(group_heads), 1)
+    n = ctypes.c_int32()
+    lo, hi = (ctypes.c_int32 * cap)(), (ctypes.c_int32 * cap)()
+    _check(_lib.usp_head_chunk_ranges(group_heads, num_chunks, ctypes.byref(n), lo, hi))
+    return [(lo[i], hi[i]) for i in range(n.value)]
+
+
+# ------------------------------------------------------------------ plan
+class Plan:
+    """Token and head ownership of `world` virtual ranks on the current device."""
+
+    def __init__(self, batch: int, seq_len: int, heads: int, head_dim: int, world: int,
+                 dtype="bf16", prefix: int = 0):
+        code = _NAMES[dtype] if isinstance(dtype, str) else _DTYPES.get(dtype, dtype)
+        handle = ctypes.c_void_p()
+        _check(_lib.usp_plan_create(ctypes.byref(handle), batch, seq_len, heads, head_dim, world, code, prefix))
+        self._h = handle
+        self.batch, self.seq_len, self.heads, self.head_dim = batch, seq_len, heads, head_dim
+        self.world, self.dtype_code, self.prefix = world, code, prefix
+        self.torch_dtype = _TORCH[code]
+        ts, tl = (ctypes.c_int64 * world)(), (ctypes.c_int64 * world)()
+        hs, hl = (ctypes.c_int32 * world)(), (ctypes.c_int32 * world)()
+        _check(_lib.usp_plan_query(self._h, ts, tl, hs, hl))
+        self.token_ranges = tuple((ts[i], ts[i] + tl[i]) for i in range(world))
+        self.head_ranges = tuple((hs[i], hs[i] + hl[i]) for i in range(world))
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise UspError(USP_ERR_INVALID_ARG, "plan is closed")
+        return self._h
+
+    @property
+    def tokens(self) -> int:
+        return self.prefix + self.seq_len
+
+    def full_shape(self):
+        return (self.batch, self.tokens, self.heads, self.head_dim)
+
+    def seq_shard_shape(self, r: int):
+        t0, t1 = self.token_ranges[r]
+        return (self.batch, self.prefix + t1 - t0, self.heads, self.head_dim)
+
+    def head_shard_shape(self, r: int):
+        h0, h1 = self.head_ranges[r]
+        return (self.batch, self.tokens, h1 - h0, self.head_dim)
+
+    def empty_seq_shards(self, dtype=None, fill=None):
+        return [self._empty(self.seq_shard_shape(r), dtype, fill) for r in range(self.world)]
+
+    def empty_head_shards(self, dtype=None, fill=None):
+        return [self._empty(self.head_shard_shape(r), dtype, fill) for r in range(self.world)]
+
+    def _empty(self, shape, dtype, fill):
+        t = torch.empty(shape, dtype=dtype or self.torch_dtype, device="cuda")
+        if fill is not None:
+            t.fill_(fill)
+        return t
+
+    def workspace_bytes(self, num_chunks: int = 1) -> int:
+        n = ctypes.c_size_t()
+        _check(_lib.usp_ulysses_attention_workspace_size(self.handle, num_chunks, ctypes.byref(n)))
+        return n.value
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.usp_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+
+def _check_tensors(plan: Plan, tensors, shapes, what: str) -> None:
+    if len(tensors) != len(shapes):
+        raise UspError(USP_ERR_INVALID_ARG, f"{what}: expected {len(shapes)} tensors, got {len(tensors)}")
+    elem = torch.empty((), dtype=plan.torch_dtype).element_size()
+    for i, (t, shape) in enumerate(zip(tensors, shapes)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise UspError(USP_ERR_INVALID_ARG, f"{what}[{i}] must be a contiguous CUDA tensor")
+        if t.element_size() != elem:
+            raise UspError(USP_ERR_DTYPE, f"{what}[{i}] has {t.element_size()}-byte elements, plan has {elem}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise UspError(USP_ERR_SHAPE, f"{what}[{i}] has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+# --------------------------------------------------------- layout operations
+def scatter_sequence(plan: Plan, x_full, out=None, stream=None):
+    """API page, scatter_sequence: per-rank token windows of a replicated tensor."""
+    out = out if out is not None else [torch.empty(plan.seq_shard_shape(r), dtype=x_full.dtype, device=x_full.device)
+                                       for r in range(plan.world)]
+    _check_tensors(plan, [x_full], [plan.full_shape()], "x_full")
+    _check_tensors(plan, out, [plan.seq_shard_shape(r) for r in range(plan.world)], "x_shards")
+    _check(_lib.usp_scatter_sequence(plan.handle, x_full.data_ptr(), _ptrs(out), 0, 0, _stream(stream)))
+    return out
+
+
+def gather_sequence(plan: Plan, shards, out=None, stream=None):
+    """API page, gather_sequence: the full tensor from the shards, in rank order."""
+    out = out if out is not None else torch.empty(plan.full_shape(), dtype=shards[0].dtype, device=shards[0].device)
+    _check_tensors(plan, shards, [plan.seq_shard_shape(r) for r in range(plan.world)], "x_shards")
+    _check_tensors(plan, [out], [plan.full_shape()], "x_full")
+    _check(_lib.usp_gather_sequence(plan.handle, _ptrs(shards), out.data_ptr(), 0, 0, _stream(stream)))
+    return out
+
+
+def sp_head_slice(plan: Plan, x_full, out=None, stream=None):
+    """API page, sp_head_slice: each rank's contiguous head group of [B, T', H, D]."""
+    out = out if out is not None else [torch.empty(plan.head_shard_shape(r), dtype=x_full.dtype, device=x_full.device)
+                                       for r in range(plan.world)]
+    _check_tensors(plan, [x_full], [plan.full_shape()], "x_full")
+    _check_tensors(plan, out, [plan.head_shard_shape(r) for r in range(plan.world)], "x_head_shards")
+    _check(_lib.usp_sp_head_slice(plan.handle, x_full.data_ptr(), _ptrs(out), 0, _stream(stream)))
+    return out
+
+
+def sp_head_gather(plan: Plan, head_shards, out=None, stream=None):
+    """API page, sp_head_gather: inverse of sp_head_slice."""
+    out = out if out is not None else torch.empty(plan.full_shape(), dtype=head_shards[0].dtype,
+                                                  device=head_shards[0].device)
+    _check_tensors(plan, head_shards, [plan.head_shard_shape(r) for r in range(plan.world)], "x_head_shards")
+    _check_tensors(plan, [out], [plan.full_shape()], "x_full")
+    _check(_lib.usp_sp_head_gather(plan.handle, _ptrs(head_shards), out.data_ptr(), 0, _stream(stream)))
+    return out
+
+
+def ulysses_seq_to_head(plan: Plan, tensors, out=None, stream=None):
+    """Ragged transport page, seq_to_heads: `tensors` is a list of 1..3 lists of
+    per-rank sequence shards (q, k, v); returns the matching per-rank head shards."""
+    n = len(tensors)
+    if out is None:
+        out = [[torch.empty(plan.head_shard_shape(r), dtype=tensors[0][0].dtype, device=tensors[0][0].device)
+                for r in range(plan.world)] for _ in range(n)]
+    flat_in = [t for group in tensors for t in group]
+    flat_out = [t for group in out for t in group]
+    _check_tensors(plan, flat_in, [plan.seq_shard_shape(r) for _ in range(n) for r in range(plan.world)], "in")
+    _check_tensors(plan, flat_out, [plan.head_shard_shape(r) for _ in range(n) for r in range(plan.world)], "out")
+    _check(_lib.usp_ulysses_seq_to_head(plan.handle, n, _ptrs(flat_in), _ptrs(flat_out), _stream(stream)))
+    return out
+
+
+def ulysses_head_to_seq(plan: Plan, tensors, out=None, stream=None):
+    """Ragged transport page, heads_to_seq: per-rank head shards back to sequence shards."""
+    n = len(tensors)
+    if out is None:
+        out = [[torch.empty(plan.seq_shard_shape(r), dtype=tensors[0][0].dtype, device=tensors[0][0].device)
+                for r in range(plan.world)] for _ in range(n)]
+    flat_in = [t for group in tensors for t in group]
+    flat_out = [t for group in out for t in group]
+    _check_tensors(plan, flat_in, [plan.head_shard_shape(r) for _ in range(n) for r in range(plan.world)], "in")
+    _check_tensors(plan, flat_out, [plan.seq_shard_shape(r) for _ in range(n) for r in range(plan.world)], "out")
+    _check(_lib.usp_ulysses_head_to_seq(plan.handle, n, _ptrs(flat_in), _ptrs(flat_out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------- attention
+def head_attention(plan: Plan, q_heads, k_heads, v_heads, out=None, scale: float = 0.0, stream=None):
+    """run_attention on every rank's head shard (non-causal softmax attention)."""
+    shapes = [plan.head_shard_shape(r) for r in range(plan.world)]
+    out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
+    for name, ts in (("q_heads", q_heads), ("k_heads", k_heads), ("v_heads", v_heads), ("o_heads", out)):
+        _check_tensors(plan, ts, shapes, name)
+    _check(_lib.usp_head_attention(plan.handle, _ptrs(q_heads), _ptrs(k_heads), _ptrs(v_heads), _ptrs(out),
+                                   float(scale), _stream(stream)))
+    return out
+
+
+def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chunks: int = 1,
+                      workspace=None, stream=None):
+    """API page, ulysses_attention (with head-chunked passes): per-rank sequence
+    shards of q, k, v in; per-rank sequence shards of the attention output out."""
+    shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
+    out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
+    for name, ts in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _check_tensors(plan, ts, shapes, name)
+    need = plan.workspace_bytes(num_chunks)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if workspace.numel() * workspace.element_size() < need:
+        raise UspError(USP_ERR_SHAPE, f"workspace needs {need} bytes")
+    _check(_lib.usp_ulysses_attention(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
+                                      num_chunks, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)))
+    return out
+
+
+def device_status(reset: bool = True) -> int:
+    """Synchronises the device and returns the library's device-side error word."""
+    code = ctypes.c_uint32()
+    rc = _lib.usp_device_status(ctypes.byref(code), 1 if reset else 0)
+    if rc not in (USP_OK, USP_ERR_TIMEOUT):
+        _check(rc)
+    return code.value
+
+
+def debug_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(_lib.usp_debug_wait_timeout(limit_us, _stream(stream)))
