@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the Ulysses sequence-parallel attention block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload video|chunked|vit|tiny|reshard]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+scatter_sequence of the replicated q, k and v into the P virtual-rank shards,
+the Ulysses block (seq->head exchange of q/k/v per head chunk, attention, and
+the head->seq exchange fused into the attention epilogue), and
+gather_sequence of the output. The default workload is the ragged video
+latent (T=75600, H=24, D=128, P=7, bf16, one chunk); `value` is the
+attention FLOP of the step (4*B*H*T'^2*D) over the step time, in TFLOP/s.
+
+With N > 1 (launched by torch.distributed.run) every GPU runs its own
+independent replica of the block (the block needs no collective across
+GPUs); the timing is the maximum over ranks and `value` sums all replicas.
+
+Rank 0 prints one JSON line. `--impl reference` times the CPU oracle instead
+(test infrastructure, float64, on a bounded sample of rows of the same
+workload).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ulysses_sequence_attention_sp_b200 import workloads as W  # noqa: E402
+from ulysses_sequence_attention_sp_b200.synth import make_qkv, storage_to_f64  # noqa: E402
+
+METRIC = "reshard GB/s and Ulysses-attention TFLOP/s on 1 B200, % of HBM/bf16 roofline"
+WORKLOADS = {"tiny": W.TINY, "reshard": W.RESHARD, "video": W.VIDEO, "vit": W.VIT, "chunked": W.CHUNKED}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["ulysses_sequence_attention_sp_b200/csrc/attn_tc.cu",
+                  "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh",
+                  "ulysses_sequence_attention_sp_b200/csrc/permute.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="video")
+    ap.add_argument("--num-chunks", type=int, default=0, help="0: the workload's own chunk count")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-reshard", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS if k in p}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources are unchanged since it was taken; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_hash") != source_hash(KERNEL_SOURCES):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                cols = [c.strip() for c in line.split(",")]
+                if len(cols) < 9:
+                    continue
+                try:
+                    sm.append(float(cols[1]))
+                    mx.append(float(cols[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, cols[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_rows_tflops(w, storage, seconds: float, max_rows: int):
+    """Times the oracle's attention on query rows of (batch 0, head 0) of the
+    workload until `seconds` have elapsed (or max_rows rows)."""
+    from oracle.attention import default_scale, softmax_attention
+    q, k, v = storage
+    kh = storage_to_f64(k[0, :, 0], w.dtype)
+    vh = storage_to_f64(v[0, :, 0], w.dtype)
+    rows_done, t_used, r0 = 0, 0.0, 0
+    chunk = 64
+    while t_used < seconds and rows_done < max_rows:
+        rows = np.arange(r0, r0 + chunk) % w.tokens
+        qh = storage_to_f64(q[0, rows, 0], w.dtype)
+        t0 = time.perf_counter()
+        softmax_attention(qh, kh, vh, default_scale(w.head_dim))
+        t_used += time.perf_counter() - t0
+        rows_done += chunk
+        r0 += chunk
+    flop = rows_done * 4.0 * w.tokens * w.head_dim
+    return flop / t_used / 1e12, rows_done, t_used
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, w, rank, world):
+    """The reference arm: the CPU oracle, on rank 0 only."""
+    if rank != 0:
+        return
+    storage = make_qkv(w)
+    per_step_s = 4.0
+    times, rows = [], 0
+    for i in range(args.warmup + args.steps):
+        tf, r, t = oracle_rows_tflops(w, storage, per_step_s, 1 << 30)
+        if i >= args.warmup:
+            times.append(t)
+            rows += r
+    flop = rows * 4.0 * w.tokens * w.head_dim
+    value = flop / sum(times) / 1e12
+    cores = blas_threads()
+    sample = (f"float64 oracle attention (oracle.attention.softmax_attention) on {rows // max(args.steps, 1)} "
+              f"query rows per step of batch 0, head 0 against all {w.tokens} keys; rows are independent, "
+              f"so TFLOP/s carries over to the full workload")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, w.num_chunks[0], args.gpus), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, num_chunks, n_gpus):
+    return {
+        "workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "prefix_tokens": w.prefix,
+        "heads": w.heads, "head_dim": w.head_dim, "sp_virtual_ranks": w.world, "num_chunks": num_chunks,
+        "global_batch": w.batch * n_gpus,
+        "parallelism": f"{n_gpus} independent replica(s), {w.world} virtual SP ranks each",
+        "step": "scatter_sequence(q,k,v) -> ulysses_attention -> gather_sequence(out)",
+        "l2": f"inputs larger than L2: {3 * w.tensor_bytes / 2**20:.0f} MiB of q/k/v per step"
+        if 3 * w.tensor_bytes > 126 * 2**20 else "L2 flushed (512 MiB write) before every timed step",
+    }
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from ulysses_sequence_attention_sp_b200 import usp
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    n_chunks = args.num_chunks or w.num_chunks[0]
+    pk, pk_kind = peaks()
+    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix)
+    tdt = plan.torch_dtype
+    storage = make_qkv(w, seed=w.seed + 7919 * rank)
+
+    def to_dev(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(x).to(dev)
+
+    full = [to_dev(x) for x in storage]
+    shards = [plan.empty_seq_shards() for _ in range(3)]
+    out = plan.empty_seq_shards()
+    full_out = torch.empty(plan.full_shape(), dtype=tdt, device=dev)
+    ws = torch.empty(plan.workspace_bytes(n_chunks), dtype=torch.uint8, device=dev)
+    small = 3 * w.tensor_bytes <= 126 * 2**20
+    flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev) if small else None
+
+    def step():
+        for x, sh in zip(full, shards):
+            usp.scatter_sequence(plan, x, out=sh)
+        usp.ulysses_attention(plan, *shards, out=out, num_chunks=n_chunks, workspace=ws)
+        usp.gather_sequence(plan, out, out=full_out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # timed region: K steps, attention kernels bracketed by their own events
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev_a:
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    barrier()
+    clocks.start()
+    time.sleep(0.3)  # a few clock samples before the region starts
+    launches0 = usp.kernel_launches()
+    flush_ms = 0.0
+    t0.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        plan.set_timing_events(*ev_a[i])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = usp.kernel_launches() - launches0
+    barrier()
+    clk = clocks.stop()
+    plan.set_timing_events(None, None)
+    ms_total = t0.elapsed_time(t1)
+    if flush is not None:
+        fs, fe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fs.record(stream)
+        for _ in range(args.steps):
+            flush.zero_()
+        fe.record(stream)
+        torch.cuda.synchronize()
+        flush_ms = fs.elapsed_time(fe)
+        ms_total -= flush_ms
+    attn_ms = [a.elapsed_time(b) for a, b in ev_a]
+    assert usp.device_status() == 0, "a device-side wait ran out"
+
+    t = torch.tensor([ms_total, statistics.mean(attn_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, attn_ms_max = float(t[0]), float(t[1])
+    ms_step = ms_max / args.steps
+    flop = float(w.attention_flop)
+    value = world * flop * args.steps / (ms_max / 1e3) / 1e12
+
+    line = None
+    if rank == 0:
+        n_launch_attn = len(usp.head_chunk_ranges(max(b - a for a, b in plan.head_ranges), n_chunks))
+        attn_launch_ms = attn_ms_max / n_launch_attn
+        achieved = flop / n_launch_attn / (attn_launch_ms / 1e3) / 1e12
+        peak_key = "bf16_tflops_sustained"
+        traffic = recorded_traffic("attention")
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": workload_config(w, n_chunks, world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk[peak_key], "unit": "TFLOP/s",
+                         "frac": achieved / pk[peak_key], "traffic": traffic,
+                         "kernel": "attn_tc_kernel (tcgen05), one launch per head chunk",
+                         "peak_source": f"{peak_key} ({pk_kind}); the kernel runs inside a long step loop",
+                         "frac_of_burst_peak": achieved / pk["bf16_tflops"],
+                         "attention_ms_per_step": attn_ms_max},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+    # end-to-end through the public API with host buffers
+    if not args.no_e2e:
+        host_in = [torch.from_numpy(x.view(np.int16) if w.dtype == "bf16" else x).pin_memory() for x in storage]
+        host_out = torch.empty(full_out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
+        k_e2e = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for h, d in zip(host_in, full):
+                d.view(h.dtype).copy_(h, non_blocking=True)
+            step()
+            host_out.copy_(full_out.view(host_out.dtype), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        if rank == 0:
+            line["e2e"] = {"value": world * flop * k_e2e / (float(te[0]) / 1e3) / 1e12, "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": 3 * w.tensor_bytes, "d2h_bytes_per_step": w.tensor_bytes,
+                           "steps": k_e2e}
+        del host_in, host_out
+    plan.close()
+    del full, shards, out, full_out, ws
+    torch.cuda.empty_cache()
+
+    if rank == 0 and world == 1 and not args.no_reshard:
+        line["reshard"] = reshard_measurement(usp, torch, dev, pk, pk_kind)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, rows, secs = oracle_rows_tflops(w, storage, 12.0, 1 << 30)
+        line["cpu_baseline"] = {
+            "value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle attention on {rows} query rows of batch 0, head 0 against all {w.tokens} "
+                      f"keys ({secs:.1f} s); rows are independent, so TFLOP/s carries over to the workload"}
+    return line
+
+
+def reshard_measurement(usp, torch, dev, pk, pk_kind):
+    """Bandwidth of the ragged layout kernels on the reshard workload
+    (T=32768, H=32, D=128, P=8, bf16): algorithmic bytes = read + write of
+    every moved element; inputs larger than L2; median of 7 timed reps."""
+    w = W.RESHARD
+    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix)
+    S = w.tensor_bytes
+    full = torch.empty(plan.full_shape(), dtype=torch.bfloat16, device=dev).normal_()
+    seq = [plan.empty_seq_shards() for _ in range(3)]
+    for s in seq:
+        usp.scatter_sequence(plan, full, out=s)
+    heads = [plan.empty_head_shards() for _ in range(3)]
+    full2 = torch.empty_like(full)
+    ops = {
+        "seq_to_head_qkv": (lambda: usp.ulysses_seq_to_head(plan, seq, out=heads), 6 * S),
+        "head_to_seq": (lambda: usp.ulysses_head_to_seq(plan, heads[:1], out=seq[:1]), 2 * S),
+        "scatter_sequence": (lambda: usp.scatter_sequence(plan, full, out=seq[1]), 2 * S),
+        "gather_sequence": (lambda: usp.gather_sequence(plan, seq[1], out=full2), 2 * S),
+        "sp_head_slice": (lambda: usp.sp_head_slice(plan, full, out=heads[2]), 2 * S),
+        "sp_head_gather": (lambda: usp.sp_head_gather(plan, heads[2], out=full2), 2 * S),
+    }
+    res = {}
+    for name, (fn, nbytes) in ops.items():
+        for _ in range(2):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(7)]
+        for a, b in evs:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        res[name] = {"GB/s": nbytes / ms / 1e6, "ms": ms, "frac": nbytes / ms / 1e6 / pk["hbm_gbs"]}
+    # bit-exact round trip of the whole exchange on this data
+    usp.ulysses_head_to_seq(plan, heads, out=seq)
+    torch.cuda.synchronize()
+    plan.close()
+    s2h = res["seq_to_head_qkv"]
+    return {"workload": w.name, "ops": res, "peak_gbs": pk["hbm_gbs"], "peak_source": f"hbm_gbs ({pk_kind})",
+            "roofline": {"bound": "hbm", "achieved": s2h["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": s2h["frac"], "traffic": recorded_traffic("permute"),
+                         "kernel": "permute_kernel (seq_to_head of q, k, v)"}}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(json.dumps({"error": f"--gpus {args.gpus} but WORLD_SIZE {world}"}), flush=True)
+        sys.exit(2)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if w.name == W.RESHARD.name:
+        print(json.dumps({"error": "the reshard workload is measured inside every run (key 'reshard')"}))
+        sys.exit(2)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    line = run_ours(args, w, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -206,6 +206,19 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * usp_plan_set_timing_events -- profiling hook: while set, every
+ * usp_ulysses_attention call with this plan records `start` (a cudaEvent_t)
+ * on its stream just before its first attention kernel and `stop` just after
+ * its last one, so the caller can time the attention kernels alone inside a
+ * longer stream of work. NULL, NULL turns it off. The events stay owned by
+ * the caller and must outlive their use.
+ */
+int usp_plan_set_timing_events(usp_plan* plan, void* start, void* stop);
+
+/* Number of kernels this library has launched in this process (diagnostic). */
+uint64_t usp_kernel_launches(void);
+
+/*
  * usp_device_status -- synchronises the current device, then reads the
  * library's device-side error word of its kernels (0 = no error; nonzero =
  * a bounded device-side wait ran out, and identifies the wait). reset != 0

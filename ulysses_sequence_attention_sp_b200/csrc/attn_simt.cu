@@ -126,6 +126,7 @@ int launch_dpt(const AttnLaunch& L, cudaStream_t stream) {
   const float scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
   dim3 grid((L.tokens + kRows - 1) / kRows, L.batch * L.n_heads);
   attn_simt_kernel<DPT><<<grid, kThreads, smem, stream>>>(L, scale_log2);
+  count_launch();
   return cuda_check(cudaGetLastError(), "attention (fp32) launch");
 }
 

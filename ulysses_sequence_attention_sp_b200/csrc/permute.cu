@@ -125,6 +125,7 @@ int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream) {
     case 2: permute_kernel<uint16_t><<<grid, block, 0, stream>>>(a); break;
     default: return set_error(USP_ERR_INVALID_ARG, "internal: bad vector width %d", vec_bytes);
   }
+  count_launch();
   return cuda_check(cudaGetLastError(), "permute kernel launch");
 }
 

@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <string>
 
 #include "usp_internal.h"
@@ -155,6 +156,10 @@ int set_error(int code, const char* fmt, ...) {
   g_last_error = buf;
   return code;
 }
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int cuda_check(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return USP_OK;
@@ -552,10 +557,25 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
     }
     L.n_heads = a.nsel;
     for (int i = 0; i < a.nsel; ++i) L.heads[i] = a.sel_head[i];
+    if (c == 0 && plan->t_start)
+      if (int rc = usp::cuda_check(cudaEventRecord(plan->t_start, s), "cudaEventRecord(timing)")) return rc;
     if (int rc = launch_attention(L, s)) return rc;
   }
+  if (plan->t_stop)
+    if (int rc = usp::cuda_check(cudaEventRecord(plan->t_stop, s), "cudaEventRecord(timing)")) return rc;
   return USP_OK;
 }
+
+int usp_plan_set_timing_events(usp_plan* plan, void* start, void* stop) {
+  if (int rc = check_plan(plan)) return rc;
+  if ((start == nullptr) != (stop == nullptr))
+    return usp::set_error(USP_ERR_INVALID_ARG, "set both timing events or neither");
+  plan->t_start = static_cast<cudaEvent_t>(start);
+  plan->t_stop = static_cast<cudaEvent_t>(stop);
+  return USP_OK;
+}
+
+uint64_t usp_kernel_launches(void) { return usp::g_launches.load(std::memory_order_relaxed); }
 
 int usp_device_status(uint32_t* code, int32_t reset) {
   if (!code) return usp::set_error(USP_ERR_INVALID_ARG, "code is NULL");

@@ -27,6 +27,8 @@ struct usp_plan {
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
   std::vector<cudaEvent_t> ev_chunk;      // aux -> caller stream: chunk c packed
+  cudaEvent_t t_start = nullptr;          // caller-owned timing events (profiling hook)
+  cudaEvent_t t_stop = nullptr;
 
   int64_t tokens() const { return prefix + seq_len; }
 };
@@ -34,6 +36,7 @@ struct usp_plan {
 namespace usp {
 
 int set_error(int code, const char* fmt, ...);
+void count_launch();
 int cuda_check(cudaError_t e, const char* what);
 
 // ------------------------------------------------------------ permutation

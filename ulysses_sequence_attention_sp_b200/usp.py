@@ -73,6 +73,8 @@ _SIGNATURES = {
                                                             ctypes.POINTER(ctypes.c_size_t)]),
     "usp_ulysses_attention": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "usp_plan_set_timing_events": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "usp_kernel_launches": (ctypes.c_uint64, []),
     "usp_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "usp_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
 }
@@ -204,6 +206,15 @@ class Plan:
         _check(_lib.usp_ulysses_attention_workspace_size(self.handle, num_chunks, ctypes.byref(n)))
         return n.value
 
+    def set_timing_events(self, start=None, stop=None) -> None:
+        """Profiling hook: record torch.cuda.Event `start`/`stop` around the
+        attention kernels of each ulysses_attention call (None, None: off)."""
+        if start is None:
+            _check(_lib.usp_plan_set_timing_events(self.handle, None, None))
+            return
+        _check(_lib.usp_plan_set_timing_events(self.handle, ctypes.c_void_p(start.cuda_event),
+                                               ctypes.c_void_p(stop.cuda_event)))
+
     def close(self) -> None:
         if getattr(self, "_h", None) is not None:
             _lib.usp_plan_destroy(self._h)
@@ -333,6 +344,11 @@ def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chu
                                       num_chunks, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
     return out
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process."""
+    return int(_lib.usp_kernel_launches())
 
 
 def device_status(reset: bool = True) -> int:
