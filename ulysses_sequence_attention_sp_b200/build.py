@@ -51,8 +51,8 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= lib_mtime for f in _deps())
 
 
-def _compile(src: str, extra: list[str], verbose: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
+def _compile(src: str, extra: list[str], verbose: bool, build_dir: str = BUILD_DIR) -> str:
+    obj = os.path.join(build_dir, os.path.splitext(src)[0] + ".o")
     cmd = [nvcc(), *ARCH, *COMMON, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
     if src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"] if verbose else []
@@ -64,22 +64,26 @@ def _compile(src: str, extra: list[str], verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compiles every source for sm_100a and links libusp.so; returns its path."""
-    if not force and not extra and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    """Compiles every source for sm_100a and links libusp.so (or `out`, for a
+    variant built with `extra` flags such as -DUSP_TRACE); returns its path."""
+    lib_path = out or LIB_PATH
+    if not force and not extra and out is None and up_to_date():
         return LIB_PATH
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    build_dir = BUILD_DIR if out is None else os.path.join(BUILD_DIR, "variant")
+    os.makedirs(build_dir, exist_ok=True)
     extra = list(extra or [])
     with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra, verbose), SOURCES))
-    tmp = LIB_PATH + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, extra, verbose, build_dir), SOURCES))
+    tmp = lib_path + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
         raise RuntimeError("linking libusp.so failed")
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main() -> None:

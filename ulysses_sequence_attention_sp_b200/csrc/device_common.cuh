@@ -215,6 +215,56 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (two lanes per instruction on sm_100).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no MUFU), x >= -125 and x < 2^22:
+// n = round(x) via the 1.5*2^23 rounding constant, f = x - n in [-1/2, 1/2],
+// 2^f by a degree-3 polynomial (Remez fit of the relative error, max 7.5e-5;
+// coefficients from csrc/fit_exp2_poly.py), and 2^n added to the exponent
+// field as an integer. Cody and Waite's argument reduction.
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t round2 = f2_pack(kRound, kRound);
+  const uint64_t neg_round2 = f2_pack(-kRound, -kRound);
+  const uint64_t t = f2_add(x, round2);            // low mantissa bits hold round(x)
+  const uint64_t n = f2_add(t, neg_round2);        // round(x) as float
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);  // x - n, exact
+  uint64_t p = f2_fma(f, f2_pack(0.055171669f, 0.055171669f), f2_pack(0.24261112f, 0.24261112f));
+  p = f2_fma(p, f, f2_pack(0.69326099f, 0.69326099f));
+  p = f2_fma(p, f, f2_pack(0.99992807f, 0.99992807f));
+  float t0, t1, p0, p1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(p, p0, p1);
+  // exponent(p) += round(x): the integer in t's low bits, shifted to bit 23
+  const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);
+  const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 // Packs two floats into bf16x2 / f16x2 with round-to-nearest-even; `lo` in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

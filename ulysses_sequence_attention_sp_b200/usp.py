@@ -83,7 +83,9 @@ EXPORTED = tuple(_SIGNATURES)
 
 
 def library_path() -> str:
-    return os.path.join(_HERE, _LIB_NAME)
+    """The in-tree libusp.so, or the build named by $USP_LIBRARY (a variant
+    built with extra flags, e.g. the pipeline-trace build)."""
+    return os.environ.get("USP_LIBRARY") or os.path.join(_HERE, _LIB_NAME)
 
 
 def _load():
