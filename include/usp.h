@@ -206,6 +206,32 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * usp_ulysses_attention_noalloc -- the source pages have no counterpart; this
+ * entry point exists for callers that cannot allocate device memory when they
+ * call the block, for example a plugin or custom operator whose host
+ * framework owns all device memory and passes only the inputs and outputs, or
+ * code on a path that must not synchronise the device (cudaFree does).
+ *
+ * It computes exactly what usp_ulysses_attention computes, with the same
+ * arguments except the workspace: its scratch is a fixed array of
+ * USP_NOALLOC_SCRATCH_BYTES inside the library's device memory, which every
+ * GPU that loads the library holds until the process exits. The call makes no
+ * cudaMalloc or cudaFree call and uses no allocating library routine.
+ *  - Plans whose usp_ulysses_attention_workspace_size exceeds the array are
+ *    rejected with USP_ERR_SHAPE before any launch.
+ *  - The first call on a device looks up the array's device address there
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Calls that overlap on the GPU (other streams, other host threads) race on
+ *    it: order them. Nothing in it has to start at zero.
+ */
+#define USP_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int usp_ulysses_attention_noalloc(const usp_plan* plan, const void* const* q, const void* const* k,
+                                  const void* const* v, void* const* out, float scale, int32_t num_chunks,
+                                  void* stream);
+
+/*
  * usp_plan_set_timing_events -- profiling hook: while set, every
  * usp_ulysses_attention call with this plan records `start` (a cudaEvent_t)
  * on its stream just before its first attention kernel and `stop` just after

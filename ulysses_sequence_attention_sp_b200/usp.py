@@ -73,6 +73,8 @@ _SIGNATURES = {
                                                             ctypes.POINTER(ctypes.c_size_t)]),
     "usp_ulysses_attention": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "usp_ulysses_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
+                                                     ctypes.c_int32, ctypes.c_void_p]),
     "usp_plan_set_timing_events": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "usp_kernel_launches": (ctypes.c_uint64, []),
     "usp_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
@@ -345,6 +347,24 @@ def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chu
     _check(_lib.usp_ulysses_attention(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
                                       num_chunks, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def ulysses_attention_noalloc(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chunks: int = 1,
+                              stream=None):
+    """ulysses_attention for callers that cannot allocate device memory: the
+    scratch is a fixed array inside the library (NOALLOC_SCRATCH_BYTES, shared by
+    all calls; calls that overlap on the GPU race). `out` must be given by such
+    a caller; when it is None this helper allocates it with torch for convenience."""
+    shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
+    out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
+    for name, ts in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _check_tensors(plan, ts, shapes, name)
+    _check(_lib.usp_ulysses_attention_noalloc(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
+                                              num_chunks, _stream(stream)))
     return out
 
 
