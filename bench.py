@@ -45,9 +45,11 @@ METRIC = "reshard GB/s and Ulysses-attention TFLOP/s on 1 B200, % of HBM/bf16 ro
 WORKLOADS = {"tiny": W.TINY, "reshard": W.RESHARD, "video": W.VIDEO, "vit": W.VIT, "chunked": W.CHUNKED}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["ulysses_sequence_attention_sp_b200/csrc/attn_tc.cu",
-                  "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh",
-                  "ulysses_sequence_attention_sp_b200/csrc/permute.cu"]
+KERNEL_SOURCES = {
+    "attention": ["ulysses_sequence_attention_sp_b200/csrc/attn_tc.cu",
+                  "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh"],
+    "permute": ["ulysses_sequence_attention_sp_b200/csrc/permute.cu"],
+}
 
 
 def parse_args():
@@ -61,6 +63,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-reshard", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every call from Python instead of replaying the step as one CUDA graph")
     return ap.parse_args()
 
 
@@ -88,7 +92,7 @@ def recorded_traffic(kernel: str):
         return None
     with open(TRAFFIC_FILE) as f:
         rec = json.load(f).get(kernel)
-    if not rec or rec.get("source_hash") != source_hash(KERNEL_SOURCES):
+    if not rec or rec.get("source_hash") != source_hash(KERNEL_SOURCES[kernel]):
         return None
     return rec.get("bytes_per_launch")
 
@@ -103,8 +107,11 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.skip = 0
 
     def start(self):
+        """Starts sampling and returns once the first sample is written, so
+        nvidia-smi's own start-up never overlaps the timed region."""
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -113,6 +120,11 @@ class ClockSampler:
                  "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        deadline = time.time() + 10.0
+        while time.time() < deadline and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+            time.sleep(0.05)
+        self.skip = sum(1 for _ in open(self.path))  # samples taken before the timed region
 
     def stop(self):
         if self.proc is None:
@@ -125,18 +137,21 @@ class ClockSampler:
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                cols = [c.strip() for c in line.split(",")]
-                if len(cols) < 9:
-                    continue
-                try:
-                    sm.append(float(cols[1]))
-                    mx.append(float(cols[2]))
-                except ValueError:
-                    continue
-                for name, val in zip(names, cols[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(name)
+            lines = f.readlines()
+        if len(lines) > self.skip + 1:
+            lines = lines[self.skip:]  # keep the samples taken during the timed region
+        for line in lines:
+            cols = [c.strip() for c in line.split(",")]
+            if len(cols) < 9:
+                continue
+            try:
+                sm.append(float(cols[1]))
+                mx.append(float(cols[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, cols[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
         os.unlink(self.path)
         if not sm:
             return None
@@ -206,6 +221,22 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def reduce_max(values, world, device=None):
+    """Element-wise maximum of per-rank timings over all ranks (any backend:
+    NCCL needs a CUDA tensor, gloo a CPU one)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device or "cpu")
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(units_per_rank_step: float, steps: int, max_ms: float, world: int, scale: float = 1e12):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3) / scale
+
+
 def workload_config(w, num_chunks, n_gpus):
     return {
         "workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "prefix_tokens": w.prefix,
@@ -260,29 +291,55 @@ def run_ours(args, w, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-
-    # timed region: K steps, attention kernels bracketed by their own events
+    # The step's calls are stream-ordered and synchronise nothing, so the whole
+    # step can be captured and replayed as a CUDA graph (this removes the host
+    # launch cost, which dominates the small workloads). One graph is captured
+    # per timed step, each with its own pair of attention timing events.
     ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for a, b in ev_a:
         a.record(stream)
         b.record(stream)
+    torch.cuda.synchronize()
+    graphs = []
+    launches_per_step = 0
+    if not args.no_graph:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        before = usp.kernel_launches()
+        with torch.cuda.stream(cap):
+            for i in range(args.steps):
+                g = torch.cuda.CUDAGraph()
+                plan.set_timing_events(*ev_a[i])
+                with torch.cuda.graph(g, stream=cap):
+                    step()
+                graphs.append(g)
+            plan.set_timing_events(None, None)
+        launches_per_step = (usp.kernel_launches() - before) // args.steps
+        stream.wait_stream(cap)
+        for _ in range(2):
+            graphs[0].replay()
+        torch.cuda.synchronize()
+
+    # timed region: K steps, attention kernels bracketed by their own events
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
+    clocks.start()
     torch.cuda.synchronize()
     barrier()
-    clocks.start()
-    time.sleep(0.3)  # a few clock samples before the region starts
     launches0 = usp.kernel_launches()
     flush_ms = 0.0
     t0.record(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.zero_()
-        plan.set_timing_events(*ev_a[i])
-        step()
+        if graphs:
+            graphs[i].replay()
+        else:
+            plan.set_timing_events(*ev_a[i])
+            step()
     t1.record(stream)
     torch.cuda.synchronize()
-    launches = usp.kernel_launches() - launches0
+    launches = usp.kernel_launches() - launches0 + launches_per_step * (args.steps if graphs else 0)
     barrier()
     clk = clocks.stop()
     plan.set_timing_events(None, None)
@@ -299,13 +356,10 @@ def run_ours(args, w, rank, world, local_rank):
     attn_ms = [a.elapsed_time(b) for a, b in ev_a]
     assert usp.device_status() == 0, "a device-side wait ran out"
 
-    t = torch.tensor([ms_total, statistics.mean(attn_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, attn_ms_max = float(t[0]), float(t[1])
+    ms_max, attn_ms_max = reduce_max([ms_total, statistics.mean(attn_ms)], world, dev)
     ms_step = ms_max / args.steps
     flop = float(w.attention_flop)
-    value = world * flop * args.steps / (ms_max / 1e3) / 1e12
+    value = job_throughput(flop, args.steps, ms_max, world)
 
     line = None
     if rank == 0:
@@ -318,7 +372,7 @@ def run_ours(args, w, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": workload_config(w, n_chunks, world),
+            "config": {**workload_config(w, n_chunks, world), "cuda_graph": bool(graphs)},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk[peak_key], "unit": "TFLOP/s",
                          "frac": achieved / pk[peak_key], "traffic": traffic,
                          "kernel": "attn_tc_kernel (tcgen05), one launch per head chunk",
@@ -337,7 +391,10 @@ def run_ours(args, w, rank, world, local_rank):
         def e2e_step():
             for h, d in zip(host_in, full):
                 d.view(h.dtype).copy_(h, non_blocking=True)
-            step()
+            if graphs:
+                graphs[0].replay()
+            else:
+                step()
             host_out.copy_(full_out.view(host_out.dtype), non_blocking=True)
 
         e2e_step()
@@ -349,14 +406,13 @@ def run_ours(args, w, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        (te_max,) = reduce_max([e0.elapsed_time(e1)], world, dev)
         if rank == 0:
-            line["e2e"] = {"value": world * flop * k_e2e / (float(te[0]) / 1e3) / 1e12, "unit": "TFLOP/s",
+            line["e2e"] = {"value": job_throughput(flop, k_e2e, te_max, world), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": 3 * w.tensor_bytes, "d2h_bytes_per_step": w.tensor_bytes,
                            "steps": k_e2e}
         del host_in, host_out
+    del graphs
     plan.close()
     del full, shards, out, full_out, ws
     torch.cuda.empty_cache()

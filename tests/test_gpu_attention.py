@@ -252,3 +252,50 @@ def test_invalid_attention_arguments(usp):
         ws = torch.empty(16, dtype=torch.uint8, device="cuda")
         with pytest.raises(usp.UspError):
             usp.ulysses_attention(plan, shards, shards, shards, workspace=ws)
+
+
+@pytest.mark.parametrize("num_chunks", [1, 3])
+def test_block_replays_from_a_cuda_graph(usp, num_chunks):
+    """The block's launches are stream-ordered and synchronise nothing, so the
+    whole call (with the auxiliary-stream chunk overlap) can be captured into a
+    CUDA graph and replayed on new inputs written into the same buffers."""
+    w = SMALL[0]
+    plan = _plan(usp, w)
+    ins = [plan.empty_seq_shards() for _ in range(3)]
+    out = plan.empty_seq_shards(fill=float("nan"))
+    ws = torch.empty(plan.workspace_bytes(num_chunks), dtype=torch.uint8, device="cuda")
+
+    def load(seed):
+        for x, dst in zip(make_qkv(w, seed), ins):
+            usp.scatter_sequence(plan, to_device(x, w.dtype), out=dst)
+
+    load(101)
+    usp.ulysses_attention(plan, *ins, out=out, num_chunks=num_chunks, workspace=ws)  # warm-up
+    torch.cuda.synchronize()
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        plan.set_timing_events(*ev)  # recorded as graph event nodes: every replay records them
+        with torch.cuda.graph(graph, stream=cap):
+            usp.ulysses_attention(plan, *ins, out=out, num_chunks=num_chunks, workspace=ws)
+        plan.set_timing_events(None, None)
+    torch.cuda.current_stream().wait_stream(cap)
+    for seed in (202, 303):
+        load(seed)
+        for o in out:
+            o.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = usp.ulysses_attention(plan, *ins, num_chunks=num_chunks)
+        torch.cuda.synchronize()
+        for a, b in zip(out, ref):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        assert ev[0].elapsed_time(ev[1]) > 0.0
+    assert usp.device_status() == 0
+    del graph
+    plan.close()

@@ -10,21 +10,30 @@
 // the Ulysses block that is the sequence shard of the rank owning the row's
 // token (the head->seq exchange, fused).
 //
-// One CTA computes one 128-row query tile of one (batch, head):
-//   warp 8      TMA producer: Q once, then K_j and V_j tiles into smem rings
-//   warp 9      TMEM allocator and MMA issuer (one thread):
-//                 S_j = Q K_j^T      (SS: both operands in smem)  -> TMEM S[j%2]
-//                 O  += P_{j-1} V_{j-1} (TS: P in TMEM, V in smem) -> TMEM O
-//   warps 0-7   softmax: warps w and w+4 own query rows 32(w%4).. (TMEM lane =
-//               row), each taking half of the key columns of a tile; online
+// One CTA computes one 128-row query tile of one (batch, head), walking the
+// keys in tiles of 256 (S = Q K^T is one M128 N256 MMA per 16 columns of D,
+// the shape that runs the tensor core at its full rate):
+//   warp 16     TMA producer: Q once; K in atom-column blocks (256 keys x one
+//               swizzle atom of D) and V in half tiles (128 keys x D), each
+//               into its own ring of shared-memory slots
+//   warp 17     TMEM allocator and MMA issuer (one thread):
+//                 S  = Q K_{j+1}^T  (SS)          -> TMEM S (issued as soon as the
+//                                                    softmax has loaded S_j)
+//                 O += P_j V_j      (TS: P in TMEM) -> TMEM O
+//               every K block / V half is released by its own commit
+//   warps 0-15  softmax: warps w, w+4, w+8, w+12 own query rows 32(w%4)..+32
+//               (TMEM lane = row), each taking 64 of the 256 key columns;
+//               partial row maxima are swapped through shared memory; online
 //               softmax in the log2 domain; O is rescaled in TMEM only when a
 //               row maximum grows by more than 2^8, otherwise the stale
 //               maximum is kept (exact: the final division uses the same
 //               maximum for numerator and denominator).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D), P0 [384,448), P1 [448,512).
+// TMEM columns: S [0,256), O [256,256+D), P [384,512) (256 keys, two per column).
 #include <cmath>
 #include <cstdio>
 #include <mutex>
+
+#include <cuda_fp16.h>
 
 #include "device_common.cuh"
 #include "usp_internal.h"
@@ -50,49 +59,58 @@ __device__ unsigned long long g_trace[kTraceEvents][kTraceTiles];
 
 namespace {
 
-constexpr int kBM = 128;  // query rows per CTA
-constexpr int kBN = 128;  // keys per tile
-constexpr int kThreads = 320;  // 8 softmax warps, TMA warp, MMA warp
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kBM = 128;                 // query rows per CTA
+constexpr int kBN = 256;                 // keys per tile
+constexpr int kParts = 4;                // softmax warps per TMEM lane quarter
+constexpr int kCols = kBN / kParts;      // key columns per softmax thread
+constexpr int kSoftmaxWarps = 4 * kParts;
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr int kVSlots = 2;               // V half-tile slots
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: only a broken pipeline waits this long
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s to let in-flight copies land on abort
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
-constexpr int kPolyEvery = 4;                      // one exp2 pair in four on the FMA pipe
+#ifndef USP_POLY_EVERY
+#define USP_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = USP_POLY_EVERY;         // 0: every exp2 on MUFU
 
 template <int D>
 struct Cfg {
   static constexpr int ATOM = (D % 64 == 0) ? 64 : ((D % 32 == 0) ? 32 : 16);  // elements per swizzle row
   static constexpr int NATOM = D / ATOM;
-  static constexpr int ROWB = ATOM * 2;               // bytes per row of one atom block
-  static constexpr int BLOCK_BYTES = kBM * ROWB;      // one atom block of a 128-row tile
-  static constexpr int TILE_BYTES = kBM * D * 2;
-  static constexpr uint32_t SBO = 8 * ROWB;           // 8-row core-matrix group stride
+  static constexpr int ROWB = ATOM * 2;                // bytes per row of one atom block
+  static constexpr uint32_t SBO = 8 * ROWB;            // 8-row core-matrix group stride
   static constexpr uint32_t LAYOUT = (ATOM == 64) ? 2u : ((ATOM == 32) ? 4u : 6u);
-  static constexpr int KSTAGES = (D <= 64) ? 4 : 3;
-  static constexpr int VSTAGES = (D <= 64) ? 4 : ((D <= 112) ? 3 : 2);
-  // Q + KSTAGES K tiles + VSTAGES V tiles, 1 KB alignment slack, barriers
-  static constexpr int SMEM_BYTES = TILE_BYTES * (1 + KSTAGES + VSTAGES) + 1024 + 2560;
+  static constexpr int Q_BYTES = kBM * D * 2;          // NATOM blocks of [128 rows][ROWB]
+  static constexpr int KUNIT_BYTES = kBN * ROWB;       // one atom block of a 256-key K tile
+  static constexpr int KSLOTS = NATOM + 1 < 2 ? 2 : NATOM + 1;
+  static constexpr int VHALF_BYTES = (kBN / 2) * D * 2;  // NATOM blocks of [128 keys][ROWB]
+  static constexpr int VBLOCK_BYTES = (kBN / 2) * ROWB;
+  static constexpr int KSTEPS_PER_ATOM = ATOM / 16;
+  static constexpr int SMEM_BYTES = Q_BYTES + KSLOTS * KUNIT_BYTES + kVSlots * VHALF_BYTES + 1024 + 5120;
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t k_full[9], k_empty[9];
+  uint64_t v_full[kVSlots], v_empty[kVSlots];
+  uint64_t s_full, s_empty, p_full, pv_done;
   uint64_t o_full, drain;
-  uint64_t xbar[4];          // partial-maximum exchange between warps w and w+4
+  uint64_t xbar[4];               // partial-maximum exchange among the four warps of a lane quarter
   uint32_t tmem_base;
   int abort;
-  float xch[2 * 2 * kBM];    // [tile parity][half][row]
+  float xch[2 * kParts * kBM];    // [tile parity][part][row]
 };
 
-static_assert(sizeof(Bars) + 8 <= 2560, "barrier block outgrew its shared-memory reservation");
+static_assert(sizeof(Bars) + 8 <= 5120, "barrier block outgrew its shared-memory reservation");
 
 struct TcParams {
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_q, tm_k, tm_v;   // boxes: Q 128 rows, K 256 rows, V 128 rows
   AttnOut out;
   int32_t tokens, batch, n_heads, pad0;
   float scale_log2;
@@ -102,6 +120,12 @@ struct TcParams {
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return bf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
+// Exact float values of a packed bf16x2 / f16x2 word (lo = bits 0-15).
+__device__ __forceinline__ float2 unpack2(uint32_t w, bool bf16) {
+  if (bf16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  return __half22float2(h);
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -109,9 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::TILE_BYTES;
-  uint8_t* sV = sK + C::KSTAGES * C::TILE_BYTES;
-  Bars* bars = reinterpret_cast<Bars*>(sV + C::VSTAGES * C::TILE_BYTES);
+  uint8_t* sK = sQ + C::Q_BYTES;
+  uint8_t* sV = sK + C::KSLOTS * C::KUNIT_BYTES;
+  Bars* bars = reinterpret_cast<Bars*>(sV + kVSlots * C::VHALF_BYTES);
   volatile int* abort_flag = &bars->abort;
 
   const int warp = threadIdx.x >> 5;
@@ -128,23 +152,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < C::KSTAGES; ++s) {
+    for (int s = 0; s < C::KSLOTS; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
-    for (int s = 0; s < C::VSTAGES; ++s) {
+    for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_empty[i], kSoftmaxThreads);
-      mbar_init(&bars->p_full[i], kSoftmaxThreads);
-      mbar_init(&bars->pv_done[i], 1);
-    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_empty, kSoftmaxThreads);
+    mbar_init(&bars->p_full, kSoftmaxThreads);
+    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&bars->xbar[q], 64);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->xbar[q], 32 * kParts);
     // An earlier launch or CTA recorded an error: this CTA does no work.
     bars->abort = (*reinterpret_cast<volatile uint32_t*>(&g_attn_error) != 0) ? 1 : 0;
     fence_mbar_init();
@@ -167,52 +189,58 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, C::TILE_BYTES);
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int a = 0; a < C::NATOM; ++a)
-        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * C::BLOCK_BYTES, a * C::ATOM, hm, qtile * kBM, b);
-      // K runs one tile ahead of V: K_{j+1} is needed (for S_{j+1}) before V_j.
-      auto load_k = [&](int j) -> bool {
-        const int st = j % C::KSTAGES;
-        if (j >= C::KSTAGES &&
-            !mbar_wait(&bars->k_empty[st], ((j / C::KSTAGES) - 1) & 1, abort_flag, &g_attn_error, 10, kWaitLimitNs))
+        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * kBM * C::ROWB, a * C::ATOM, hm, qtile * kBM, b);
+      // Unit n of K is atom block n % NATOM of key tile n / NATOM; half m of V is
+      // keys [128(m%2), +128) of tile m / 2. Both are issued in the order the
+      // tensor core consumes them: K of tile j+1 before V of tile j.
+      auto load_k = [&](int n) -> bool {
+        const int st = n % C::KSLOTS;
+        if (n >= C::KSLOTS &&
+            !mbar_wait(&bars->k_empty[st], ((n / C::KSLOTS) - 1) & 1, abort_flag, &g_attn_error, 10, kWaitLimitNs))
           return false;
-        mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
-        for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hm,
-                      j * kBN, b);
+        mbar_arrive_expect_tx(&bars->k_full[st], C::KUNIT_BYTES);
+        const int a = n % C::NATOM;
+        tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hm, (n / C::NATOM) * kBN, b);
         return true;
       };
-      auto load_v = [&](int j) -> bool {
-        const int st = j % C::VSTAGES;
-        if (j >= C::VSTAGES &&
-            !mbar_wait(&bars->v_empty[st], ((j / C::VSTAGES) - 1) & 1, abort_flag, &g_attn_error, 11, kWaitLimitNs))
+      auto load_v = [&](int m) -> bool {
+        const int st = m % kVSlots;
+        if (m >= kVSlots &&
+            !mbar_wait(&bars->v_empty[st], ((m / kVSlots) - 1) & 1, abort_flag, &g_attn_error, 11, kWaitLimitNs))
           return false;
-        mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
+        mbar_arrive_expect_tx(&bars->v_full[st], C::VHALF_BYTES);
         for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hm,
-                      j * kBN, b);
+          tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::VHALF_BYTES + a * C::VBLOCK_BYTES, a * C::ATOM, hm,
+                      (m / 2) * kBN + (m % 2) * (kBN / 2), b);
         return true;
       };
-      int nk = 0, nv = 0;  // tiles issued
-      if (load_k(0)) {
-        nk = 1;
-        for (int j = 0; j < ntiles; ++j) {
-          if (j + 1 < ntiles) {
-            if (!load_k(j + 1)) break;
-            nk = j + 2;
-            USP_TRACE_EV(0, j + 1);
+      int nk = 0, nv = 0;  // units issued
+      bool go = true;
+      for (int a = 0; go && a < C::NATOM; ++a) {
+        go = load_k(nk);
+        nk += go;
+      }
+      for (int j = 0; go && j < ntiles; ++j) {
+        if (j + 1 < ntiles)
+          for (int a = 0; go && a < C::NATOM; ++a) {
+            go = load_k(nk);
+            nk += go;
           }
-          if (!load_v(j)) break;
-          nv = j + 1;
-          USP_TRACE_EV(1, j);
+        USP_TRACE_EV(0, j + 1);
+        for (int h = 0; go && h < 2; ++h) {
+          go = load_v(nv);
+          nv += go;
         }
+        USP_TRACE_EV(1, j);
       }
       if (*abort_flag) {
         // Let the copies this thread started land before the CTA exits.
-        for (int j = (nk > C::KSTAGES ? nk - C::KSTAGES : 0); j < nk; ++j)
-          mbar_wait_drain(&bars->k_full[j % C::KSTAGES], (j / C::KSTAGES) & 1, kDrainLimitNs);
-        for (int j = (nv > C::VSTAGES ? nv - C::VSTAGES : 0); j < nv; ++j)
-          mbar_wait_drain(&bars->v_full[j % C::VSTAGES], (j / C::VSTAGES) & 1, kDrainLimitNs);
+        for (int n = (nk > C::KSLOTS ? nk - C::KSLOTS : 0); n < nk; ++n)
+          mbar_wait_drain(&bars->k_full[n % C::KSLOTS], (n / C::KSLOTS) & 1, kDrainLimitNs);
+        for (int m = (nv > kVSlots ? nv - kVSlots : 0); m < nv; ++m)
+          mbar_wait_drain(&bars->v_full[m % kVSlots], (m / kVSlots) & 1, kDrainLimitNs);
         mbar_wait_drain(&bars->q_full, 0, kDrainLimitNs);
       }
     }
@@ -225,44 +253,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, &g_attn_error, 20, kWaitLimitNs);
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i % C::VSTAGES;
-        if (!mbar_wait(&bars->v_full[st], (i / C::VSTAGES) & 1, abort_flag, &g_attn_error, 21, kWaitLimitNs)) return false;
-        if (!mbar_wait(&bars->p_full[i & 1], (i >> 1) & 1, abort_flag, &g_attn_error, 22, kWaitLimitNs)) return false;
-        USP_TRACE_EV(3, i);
-        tc_fence_after();
-        const uint32_t pcol = tmem + ((i & 1) ? kColP1 : kColP0);
+      tc_fence_after();
+      // S = Q K_j^T, one K atom block at a time, each block released by its own commit.
+      auto issue_qk = [&](int j) -> bool {
+        for (int a = 0; a < C::NATOM; ++a) {
+          const int n = j * C::NATOM + a;
+          const int st = n % C::KSLOTS;
+          if (!mbar_wait(&bars->k_full[st], (n / C::KSLOTS) & 1, abort_flag, &g_attn_error, 23, kWaitLimitNs))
+            return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = make_smem_desc(v_addr + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::BLOCK_BYTES,
-                                                C::SBO, C::LAYOUT);
-          umma_ts(tmem + kColO, pcol + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int ks = 0; ks < C::KSTEPS_PER_ATOM; ++ks) {
+            const uint32_t qoff = a * kBM * C::ROWB + ks * 32;
+            const uint64_t adesc = make_smem_desc(q_addr + qoff, 16, C::SBO, C::LAYOUT);
+            const uint64_t bdesc = make_smem_desc(k_addr + st * C::KUNIT_BYTES + ks * 32, 16, C::SBO, C::LAYOUT);
+            umma_ss(tmem + kColS, adesc, bdesc, idesc_qk, (a > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->k_empty[st]);
         }
-        umma_commit(&bars->pv_done[i & 1]);
-        USP_TRACE_EV(4, i);
-        umma_commit(&bars->v_empty[st]);
+        umma_commit(&bars->s_full);
+        USP_TRACE_EV(2, j);
         return true;
       };
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j % C::KSTAGES;
-        if (!mbar_wait(&bars->k_full[st], (j / C::KSTAGES) & 1, abort_flag, &g_attn_error, 23, kWaitLimitNs)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&bars->s_empty[j & 1], ((j - 2) >> 1) & 1, abort_flag, &g_attn_error, 24, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t scol = tmem + ((j & 1) ? kColS1 : kColS0);
+      // O += P_j V_j, one V half (128 keys) at a time.
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(&bars->p_full, j & 1, abort_flag, &g_attn_error, 22, kWaitLimitNs)) return false;
+        USP_TRACE_EV(3, j);
+        for (int h = 0; h < 2; ++h) {
+          const int m = 2 * j + h;
+          const int st = m % kVSlots;
+          if (!mbar_wait(&bars->v_full[st], (m / kVSlots) & 1, abort_flag, &g_attn_error, 21, kWaitLimitNs))
+            return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int e = kk * 16;
-          const uint32_t off = (e / C::ATOM) * C::BLOCK_BYTES + (e % C::ATOM) * 2;
-          const uint64_t adesc = make_smem_desc(q_addr + off, 16, C::SBO, C::LAYOUT);
-          const uint64_t bdesc = make_smem_desc(k_addr + st * C::TILE_BYTES + off, 16, C::SBO, C::LAYOUT);
-          umma_ss(scol, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 32; ++kk) {
+            const uint64_t bdesc = make_smem_desc(v_addr + st * C::VHALF_BYTES + kk * 16 * C::ROWB, C::VBLOCK_BYTES,
+                                                  C::SBO, C::LAYOUT);
+            umma_ts(tmem + kColO, tmem + kColP + h * (kBN / 4) + kk * 8, bdesc, idesc_pv, (j > 0 || h > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->v_empty[st]);
         }
-        umma_commit(&bars->s_full[j & 1]);
-        USP_TRACE_EV(2, j);
-        umma_commit(&bars->k_empty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        umma_commit(&bars->pv_done);
+        USP_TRACE_EV(4, j);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles) {
+          // S is single-buffered: the next product waits until the softmax has read S_j.
+          if (!mbar_wait(&bars->s_empty, j & 1, abort_flag, &g_attn_error, 24, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          if (!issue_qk(j + 1)) { ok = false; break; }
+        }
+        if (!issue_pv(j)) { ok = false; break; }
       }
-      if (ok) ok = issue_pv(ntiles - 1);
       if (ok) umma_commit(&bars->o_full);
       // All MMAs this thread issued must finish before TMEM is released.
       umma_commit(&bars->drain);
@@ -270,44 +314,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------- softmax
-    // Warps w and w+4 share TMEM lane quarter w%4 (32 query rows, one per
-    // thread); warp w takes key columns [0, 64) of each tile and warp w+4
-    // columns [64, 128). The two swap partial row maxima through shared
-    // memory (exchange barrier per pair), keep separate partial row sums, and
-    // split the O columns for the rescale and the epilogue.
     const int quarter = warp & 3;
-    const int half = warp >> 2;                      // 0 or 1
+    const int part = warp >> 2;                      // 0..kParts-1: key columns [kCols*part, +kCols)
     const int row = quarter * 32 + lane;             // TMEM lane = query row in the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    constexpr int kHalf = kBN / 2;                   // key columns per thread
-    constexpr int kOChunks = D / 16;
-    constexpr int kOChunks0 = (kOChunks + 1) / 2;    // O chunks of half 0
-    const int oc_lo = half ? kOChunks0 : 0;
-    const int oc_hi = half ? kOChunks : kOChunks0;
-    float* xch = bars->xch;                          // [2 parity][2 half][128 rows]
+    constexpr int kOChunks = D / 16;                 // O chunk c belongs to part c % kParts
+    float* xch = bars->xch;                          // [parity][part][row]
     uint64_t* xbar = &bars->xbar[quarter];
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // running maximum, log2 domain (identical in both halves)
-    float l = 0.f;        // this half's running denominator
+    float m = -INFINITY;  // running maximum, log2 domain (identical in the four parts)
+    float l = 0.f;        // this part's running denominator
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, &g_attn_error, 30, kWaitLimitNs))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, &g_attn_error, 30, kWaitLimitNs))) { ok = false; break; }
       if (threadIdx.x == 0) USP_TRACE_EV(5, j);
       tc_fence_after();
-      uint32_t sr[kHalf];
-      const uint32_t scol = lane_addr + ((j & 1) ? kColS1 : kColS0) + half * kHalf;
-      tmem_ld32(scol, sr);
-      tmem_ld32(scol + 32, sr + 32);
+      uint32_t sr[kCols];
+      const uint32_t scol = lane_addr + kColS + part * kCols;
+#pragma unroll
+      for (int c = 0; c < kCols; c += 32) tmem_ld32(scol + c, sr + c);
       tmem_wait_ld();
       if (threadIdx.x == 0) USP_TRACE_EV(6, j);
       tc_fence_before();
-      mbar_arrive(&bars->s_empty[j & 1]);
+      mbar_arrive(&bars->s_empty);
 
       float* s = reinterpret_cast<float*>(sr);
-      const int valid = T - j * kBN - half * kHalf;  // valid columns of this half
-      if (valid < kHalf) {
+      const int valid = T - j * kBN - part * kCols;  // valid columns of this part
+      if (valid < kCols) {
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c)
+        for (int c = 0; c < kCols; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
       // Partial row maximum: four independent three-input chains, then a tree.
@@ -316,27 +351,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int i = 0; i < 4; ++i) {
         float a = fmaxf(s[i], s[i + 4]);
 #pragma unroll
-        for (int c = i + 8; c < kHalf; c += 8) a = max3(a, s[c], s[c + 4]);
+        for (int c = i + 8; c < kCols; c += 8) a = max3(a, s[c], s[c + 4]);
         mx4[i] = a;
       }
       const float pm = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
-      // Swap partial maxima with the partner warp.
-      xch[((j & 1) * 2 + half) * kBM + row] = pm;
+      // Swap partial maxima with the other three parts of this lane quarter.
+      float* xrow = xch + (j & 1) * kParts * kBM + row;
+      xrow[part * kBM] = pm;
       mbar_arrive(xbar);
       if (!__all_sync(0xffffffffu, mbar_wait(xbar, j & 1, abort_flag, &g_attn_error, 34, kWaitLimitNs))) { ok = false; break; }
-      const float mx = fmaxf(pm, xch[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
+      const float mx = max3(fmaxf(xrow[0], xrow[kBM]), xrow[2 * kBM], xrow[3 * kBM]);
       if (threadIdx.x == 0) USP_TRACE_EV(7, j);
       const float m_new = fmaxf(m, mx * sl2);
       if (j == 0) {
         m = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
         // O holds sum_{i<j} exp2(s_i - m) v_i; bring it to the new maximum.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, &g_attn_error, 31, kWaitLimitNs))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (j - 1) & 1, abort_flag, &g_attn_error, 31, kWaitLimitNs))) { ok = false; break; }
         tc_fence_after();
         const float alpha = ex2_approx(m - m_new);
         m = m_new;
         l *= alpha;
-        for (int c = oc_lo; c < oc_hi; ++c) {
+        for (int c = part; c < kOChunks; c += kParts) {
           uint32_t o[16];
           tmem_ld16(lane_addr + kColO + c * 16, o);
           tmem_wait_ld();
@@ -347,68 +383,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tmem_wait_st();
       }
       // p = 2^(s*scale*log2e - m), packed to the input type for the P.V product.
-      // On full halves one pair in kPolyEvery takes the FMA-pipe exp2 so that
-      // the MUFU pipe is not the only exp unit; masked halves use MUFU only, so
-      // masked entries are exactly 0.
-      uint32_t pk[kHalf / 2];
-      uint64_t acc[4] = {0, 0, 0, 0};
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-m, -m);
-      if (valid >= kHalf) {
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 2) {
-          const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2);
-          float x0, x1;
-          f2_unpack(x, x0, x1);
-          uint64_t pp;
-          if ((c / 2) % kPolyEvery == kPolyEvery - 1)
-            pp = exp2_poly_f2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
-          else
-            pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], pp);
-          float p0, p1;
-          f2_unpack(pp, p0, p1);
-          pk[c / 2] = pack2(p0, p1, BF16);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 2) {
-          const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2);
-          float x0, x1;
-          f2_unpack(x, x0, x1);
-          const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          acc[(c / 2) & 3] = f2_add(acc[(c / 2) & 3], pp);
-          float p0, p1;
-          f2_unpack(pp, p0, p1);
-          pk[c / 2] = pack2(p0, p1, BF16);
-        }
-      }
+      // Masked entries (s = -inf) give exactly 0.
+      uint32_t pk[kCols / 2];
+      float psum;
       {
-        const uint64_t a01 = f2_add(acc[0], acc[1]);
-        const uint64_t a23 = f2_add(acc[2], acc[3]);
-        float u0, u1;
-        f2_unpack(f2_add(a01, a23), u0, u1);
-        l += u0 + u1;
+        // Scalar FFMA / MUFU / FADD per element. Built with USP_POLY_EVERY=n > 0,
+        // on full parts one pair in n goes through the FMA-pipe polynomial
+        // instead of MUFU (measured no faster here, so off by default).
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float negm = -m;
+        if (valid >= kCols) {
+#pragma unroll
+          for (int c = 0; c < kCols; c += 2) {
+            const float x0 = fmaf(s[c], sl2, negm);
+            const float x1 = fmaf(s[c + 1], sl2, negm);
+            float p0, p1;
+            if (kPolyEvery > 0 && (c / 2) % kPolyEvery == kPolyEvery - 1) {
+              f2_unpack(exp2_poly_f2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            acc[c & 7] += p0;
+            acc[(c + 1) & 7] += p1;
+            pk[c / 2] = pack2(p0, p1, BF16);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kCols; c += 2) {
+            const float p0 = ex2_approx(fmaf(s[c], sl2, negm));
+            const float p1 = ex2_approx(fmaf(s[c + 1], sl2, negm));
+            acc[c & 7] += p0;
+            acc[(c + 1) & 7] += p1;
+            pk[c / 2] = pack2(p0, p1, BF16);
+          }
+        }
+        psum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       }
-      // P buffer j%2 was last read by P_{j-2} V_{j-2}.
+      l += psum;
       if (threadIdx.x == 0) USP_TRACE_EV(8, j);
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, &g_attn_error, 32, kWaitLimitNs))) { ok = false; break; }
+      // P is single-buffered: it was last read by P_{j-1} V_{j-1}.
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (j - 1) & 1, abort_flag, &g_attn_error, 32, kWaitLimitNs))) { ok = false; break; }
       tc_fence_after();
-      tmem_st32(lane_addr + ((j & 1) ? kColP1 : kColP0) + half * (kHalf / 2), pk);
+      tmem_st32(lane_addr + kColP + part * (kCols / 2), pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[j & 1]);
+      mbar_arrive(&bars->p_full);
       if (threadIdx.x == 0) USP_TRACE_EV(9, j);
     }
-    // Combine the two halves' denominators.
+    // Combine the four parts' denominators.
     if (ok) {
-      xch[((ntiles & 1) * 2 + half) * kBM + row] = l;
+      float* xrow = xch + (ntiles & 1) * kParts * kBM + row;
+      xrow[part * kBM] = l;
       mbar_arrive(xbar);
       ok = __all_sync(0xffffffffu, mbar_wait(xbar, ntiles & 1, abort_flag, &g_attn_error, 35, kWaitLimitNs));
+      if (ok) l = (xrow[0] + xrow[kBM]) + (xrow[2 * kBM] + xrow[3 * kBM]);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort_flag, &g_attn_error, 33, kWaitLimitNs))) {
       tc_fence_after();
-      const float inv_l = 1.f / (l + xch[((ntiles & 1) * 2 + (half ^ 1)) * kBM + row]);
+      const float inv_l = 1.f / l;
       const int t = qtile * kBM + row;
       const AttnOut& out = p.out;
       // Destination(s) of this row.
@@ -421,14 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           row_in_seg = t;
         } else {
           const int64_t tok = t - out.prefix;
-          int s = 0;
-          while (s + 1 < out.nseg && tok >= out.seg_start[s + 1]) ++s;
-          seg_lo = s;
-          seg_hi = s + 1;
-          row_in_seg = out.prefix + tok - out.seg_start[s];
+          int sg = 0;
+          while (sg + 1 < out.nseg && tok >= out.seg_start[sg + 1]) ++sg;
+          seg_lo = sg;
+          seg_hi = sg + 1;
+          row_in_seg = out.prefix + tok - out.seg_start[sg];
         }
       }
-      for (int c = oc_lo; c < oc_hi; ++c) {
+      for (int c = part; c < kOChunks; c += kParts) {
         uint32_t o[16];
         tmem_ld16(lane_addr + kColO + c * 16, o);
         tmem_wait_ld();
@@ -478,7 +511,7 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-int make_map(CUtensorMap* map, const void* base, const AttnLaunch& L, int atom) {
+int make_map(CUtensorMap* map, const void* base, const AttnLaunch& L, int atom, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return set_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int e = 2;
@@ -486,7 +519,7 @@ int make_map(CUtensorMap* map, const void* base, const AttnLaunch& L, int atom) 
                         static_cast<cuuint64_t>(L.tokens), static_cast<cuuint64_t>(L.batch)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(L.in.stride_head * e), static_cast<cuuint64_t>(L.in.stride_token * e),
                            static_cast<cuuint64_t>(L.in.stride_batch * e)};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(atom), 1, kBM, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(atom), 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUtensorMapSwizzle swz = atom == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                       : (atom == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -511,9 +544,9 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   TcParams p;
   memset(&p, 0, sizeof(p));
   int rc;
-  if ((rc = make_map(&p.tm_q, L.in.q, L, C::ATOM)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_k, L.in.k, L, C::ATOM)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_v, L.in.v, L, C::ATOM)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_q, L.in.q, L, C::ATOM, kBM)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_k, L.in.k, L, C::ATOM, kBN)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_v, L.in.v, L, C::ATOM, kBN / 2)) != USP_OK) return rc;
   p.out = L.out;
   p.tokens = L.tokens;
   p.batch = L.batch;

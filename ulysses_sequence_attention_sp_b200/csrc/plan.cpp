@@ -453,6 +453,16 @@ int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const v
   return USP_OK;
 }
 
+// Records a caller's timing event. Under stream capture it is recorded as an
+// external event node, so every replay of the graph records it again.
+static int record_timing_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus status = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &status);
+  if (e != cudaSuccess) return usp::cuda_check(e, "cudaStreamIsCapturing");
+  const unsigned flags = status == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+  return usp::cuda_check(cudaEventRecordWithFlags(ev, s, flags), "cudaEventRecordWithFlags(timing)");
+}
+
 static size_t workspace_tensor_bytes(const usp_plan* plan) {
   const size_t bytes = static_cast<size_t>(plan->batch) * plan->tokens() * plan->heads * plan->head_dim * plan->elem;
   return (bytes + 255) & ~size_t(255);
@@ -558,11 +568,11 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
     L.n_heads = a.nsel;
     for (int i = 0; i < a.nsel; ++i) L.heads[i] = a.sel_head[i];
     if (c == 0 && plan->t_start)
-      if (int rc = usp::cuda_check(cudaEventRecord(plan->t_start, s), "cudaEventRecord(timing)")) return rc;
+      if (int rc = record_timing_event(plan->t_start, s)) return rc;
     if (int rc = launch_attention(L, s)) return rc;
   }
   if (plan->t_stop)
-    if (int rc = usp::cuda_check(cudaEventRecord(plan->t_stop, s), "cudaEventRecord(timing)")) return rc;
+    if (int rc = record_timing_event(plan->t_stop, s)) return rc;
   return USP_OK;
 }
 
