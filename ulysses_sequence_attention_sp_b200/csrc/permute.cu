@@ -9,8 +9,8 @@
 //   scatter / gather of the sequence, head slice / gather (API page)
 // The kernel walks the sequence-side rows, so that side is read or written in
 // full contiguous rows; each head unit is a contiguous run of D*elem bytes on
-// the head side. One warp moves one row at a time with vector loads of
-// 2..16 bytes, all loads of a batch issued before their stores.
+// the head side. A warp moves one segment of a row at a time (32 lanes x 4
+// vectors of 2..16 bytes), all loads of a segment issued before its stores.
 #include <cstdio>
 
 #include "device_common.cuh"
@@ -22,8 +22,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 
-template <typename V>
-__global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant__ PermuteArgs a) {
+template <typename V, int kUnitBatches>
+__global__ void __launch_bounds__(kThreads, 4) permute_kernel(const __grid_constant__ PermuteArgs a) {
   __shared__ int32_t s_unit[USP_MAX_HEADS];    // head unit index on the sequence side
   __shared__ int32_t s_rank[USP_MAX_HEADS];    // head-side buffer
   __shared__ int32_t s_local[USP_MAX_HEADS];   // unit index inside that buffer
@@ -43,8 +43,17 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
   const int64_t total_rows = a.seq_rows[a.n_seq];
   const int nvec = a.nsel * a.dv;
+  // Work is dealt out in segments of a row (kUnitBatches unrolled batches of
+  // 32 * kUnroll vectors) rather than whole rows, so the last round of the
+  // grid-stride loop is nearly full even when there are few rows per warp.
+  constexpr int kBatch = 32 * kUnroll;
+  constexpr int kSeg = kBatch * kUnitBatches;
+  const int nseg = (nvec + kSeg - 1) / kSeg;
+  const int64_t total_units = total_rows * nseg;
 
-  for (int64_t row = warp; row < total_rows; row += nwarps) {
+  for (int64_t unit = warp; unit < total_units; unit += nwarps) {
+    const int64_t row = unit / nseg;
+    const int seg = static_cast<int>(unit - row * nseg);
     int s = 0;
     while (a.seq_rows[s + 1] <= row) ++s;
     const int64_t rr = row - a.seq_rows[s];
@@ -57,14 +66,15 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant
     const int64_t t = (tl < a.prefix) ? tl : a.prefix + a.tok_start[s] + (tl - a.prefix);
     const int64_t seq_base = rr * a.heads * a.dv;
 
-    for (int j0 = 0; j0 < nvec; j0 += 32 * kUnroll) {
+    const int j_end = min(nvec, (seg + 1) * kSeg);
+    for (int j0 = seg * kSeg; j0 < j_end; j0 += kBatch) {
       int64_t soff[kUnroll], hoff[kUnroll];
       int hr[kUnroll];
       bool ok[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int j = j0 + u * 32 + lane;
-        ok[u] = j < nvec;
+        ok[u] = j < j_end;
         const int k = ok[u] ? j / a.dv : 0;
         const int d = j - k * a.dv;
         const int64_t hl = s_local[k];
@@ -110,19 +120,38 @@ int sm_count() {
 
 }  // namespace
 
-int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream) {
+int launch_permute(const PermuteArgs& args, int vec_bytes, cudaStream_t stream) {
+  PermuteArgs a = args;
   const int64_t rows = a.seq_rows[a.n_seq];
   if (rows == 0 || a.nsel == 0) return USP_OK;
-  const int64_t warps_needed = rows;
+  // Several tensors per launch already make the launch long next to its tail:
+  // deal out longer segments there to save per-segment index arithmetic.
+  a.unit_batches = a.ntensors > 1 ? 4 : 1;
+  const int64_t nvec = static_cast<int64_t>(a.nsel) * a.dv;
+  const int64_t seg = 32 * kUnroll * a.unit_batches;
+  const int64_t warps_needed = rows * ((nvec + seg - 1) / seg);
   int64_t blocks = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 resident CTAs of 256 threads per SM
   if (blocks > cap) blocks = cap;
   dim3 grid(static_cast<unsigned>(blocks)), block(kThreads);
+  const bool multi = a.unit_batches > 1;
   switch (vec_bytes) {
-    case 16: permute_kernel<uint4><<<grid, block, 0, stream>>>(a); break;
-    case 8: permute_kernel<uint2><<<grid, block, 0, stream>>>(a); break;
-    case 4: permute_kernel<uint32_t><<<grid, block, 0, stream>>>(a); break;
-    case 2: permute_kernel<uint16_t><<<grid, block, 0, stream>>>(a); break;
+    case 16:
+      if (multi) permute_kernel<uint4, 4><<<grid, block, 0, stream>>>(a);
+      else permute_kernel<uint4, 1><<<grid, block, 0, stream>>>(a);
+      break;
+    case 8:
+      if (multi) permute_kernel<uint2, 4><<<grid, block, 0, stream>>>(a);
+      else permute_kernel<uint2, 1><<<grid, block, 0, stream>>>(a);
+      break;
+    case 4:
+      if (multi) permute_kernel<uint32_t, 4><<<grid, block, 0, stream>>>(a);
+      else permute_kernel<uint32_t, 1><<<grid, block, 0, stream>>>(a);
+      break;
+    case 2:
+      if (multi) permute_kernel<uint16_t, 4><<<grid, block, 0, stream>>>(a);
+      else permute_kernel<uint16_t, 1><<<grid, block, 0, stream>>>(a);
+      break;
     default: return set_error(USP_ERR_INVALID_ARG, "internal: bad vector width %d", vec_bytes);
   }
   count_launch();

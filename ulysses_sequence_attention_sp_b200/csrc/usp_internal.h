@@ -54,7 +54,7 @@ struct PermuteArgs {
   int32_t dv;           // vectors per head unit
   int32_t head_layout;  // 0: [outer][full_tokens][C_r][dv]; 1: [C_r][outer][full_tokens][dv]
   int32_t nsel;         // head units moved (a head chunk selects a subset)
-  int32_t pad0;
+  int32_t unit_batches; // unrolled batches of a row per work unit (set by launch_permute)
   int64_t outer;        // batch
   int64_t full_tokens;  // rows per batch element on the head side (prefix + T)
   int64_t seq_rows[USP_MAX_WORLD + 1];  // prefix sums of outer * (prefix + T_s)
