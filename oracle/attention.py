@@ -12,6 +12,8 @@ Sources:
 * "maxdiffusion PR #428: experimental two-phase (head-chunked) Ulysses
   all-to-all": the head-chunked passes compute the same result as the
   single-shot pass because heads are independent.
+* API page, ulysses_attention: q carries Hq heads and k/v carry Hkv heads
+  (grouped-query attention); each kv head serves Hq / Hkv query heads.
 
 Readings: the attention is ``softmax(Q K^T * scale) V`` per (batch, head)
 with ``scale = 1/sqrt(D)`` unless given, no mask, no dropout; it is computed
@@ -26,7 +28,7 @@ import math
 import numpy as np
 
 from .layout import head_to_seq, seq_to_head
-from .partition import head_chunk_ranges, range_lengths
+from .partition import check_gqa_ranges, gqa_group, head_chunk_ranges, range_lengths
 
 # Query rows per matmul. Rows are independent, so this only bounds memory.
 _ROW_BLOCK = 512
@@ -58,16 +60,23 @@ def softmax_attention(q, k, v, scale):
 
 
 def attention_bshd(q, k, v, scale=None):
-    """Attention over ``[B, T, Hs, D]`` head-layout arrays; float64 result."""
-    if q.shape != k.shape or q.shape != v.shape:
-        raise ValueError("q/k/v must share one shape")
+    """Attention over ``[B, T, Hs, D]`` head-layout arrays; float64 result.
+
+    k and v may carry fewer heads than q (grouped-query attention, the API
+    page's Hkv <= Hq): query head h then uses kv head h // (Hq / Hkv).
+    """
+    if k.shape != v.shape or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("incompatible q/k/v shapes")
     batch, _tokens, heads, head_dim = q.shape
+    group = heads // k.shape[2]
+    if group * k.shape[2] != heads:
+        raise ValueError("query heads must be a multiple of kv heads")
     if scale is None:
         scale = default_scale(head_dim)
     out = np.empty(q.shape, dtype=np.float64)
     for b in range(batch):
         for h in range(heads):
-            out[b, :, h, :] = softmax_attention(q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], scale)
+            out[b, :, h, :] = softmax_attention(q[b, :, h, :], k[b, :, h // group, :], v[b, :, h // group, :], scale)
     return out
 
 
@@ -82,17 +91,25 @@ def attention_rows(q_full, k_full, v_full, b, h, rows, scale=None):
 
 
 def ulysses_attention(q_shards, k_shards, v_shards, token_ranges, head_ranges, *,
-                      num_chunks=1, scale=None, prefix=0):
+                      kv_head_ranges=None, num_chunks=1, scale=None, prefix=0):
     """The Ulysses block on per-rank sequence shards ``[B, prefix+T_i, H, D]``.
 
     Returns per-rank sequence shards of the float64 attention output. The
     steps are the block's: seq->head exchange of q, k and v; for each head
     chunk, attention of every rank over its heads of that chunk; head->seq
-    exchange of the output.
+    exchange of the output. With grouped-query attention k and v carry Hkv
+    heads split by ``kv_head_ranges``; query head h uses kv head
+    h // (Hq / Hkv), which must be one of its rank's kv heads.
     """
+    if kv_head_ranges is None:
+        kv_head_ranges = head_ranges
+    heads_q = head_ranges[-1][1]
+    heads_kv = kv_head_ranges[-1][1]
+    group = gqa_group(heads_q, heads_kv)
+    check_gqa_ranges(head_ranges, kv_head_ranges, group)
     qh = seq_to_head(q_shards, token_ranges, head_ranges, prefix=prefix)
-    kh = seq_to_head(k_shards, token_ranges, head_ranges, prefix=prefix)
-    vh = seq_to_head(v_shards, token_ranges, head_ranges, prefix=prefix)
+    kh = seq_to_head(k_shards, token_ranges, kv_head_ranges, prefix=prefix)
+    vh = seq_to_head(v_shards, token_ranges, kv_head_ranges, prefix=prefix)
     head_dim = q_shards[0].shape[3]
     if scale is None:
         scale = default_scale(head_dim)
@@ -100,10 +117,10 @@ def ulysses_attention(q_shards, k_shards, v_shards, token_ranges, head_ranges, *
     oh = [np.full(x.shape, np.nan, dtype=np.float64) for x in qh]
     for lo, hi in head_chunk_ranges(max(counts), num_chunks):
         for r, count in enumerate(counts):
-            a, b = min(lo, count), min(hi, count)
-            if a == b:
-                continue
-            oh[r][:, :, a:b, :] = attention_bshd(
-                qh[r][:, :, a:b, :], kh[r][:, :, a:b, :], vh[r][:, :, a:b, :], scale
-            )
+            h0, k0 = head_ranges[r][0], kv_head_ranges[r][0]
+            for i in range(min(lo, count), min(hi, count)):
+                kv = (h0 + i) // group - k0   # this rank's local kv head for local query head i
+                oh[r][:, :, i:i + 1, :] = attention_bshd(
+                    qh[r][:, :, i:i + 1, :], kh[r][:, :, kv:kv + 1, :], vh[r][:, :, kv:kv + 1, :], scale
+                )
     return head_to_seq(oh, token_ranges, head_ranges, prefix=prefix)

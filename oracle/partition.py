@@ -97,3 +97,22 @@ def rank_chunk_heads(head_ranges, num_chunks: int) -> list[list[tuple[int, int]]
             per_rank.append((h0 + a, h0 + b))
         out.append(per_rank)
     return out
+
+
+def gqa_group(heads_q: int, heads_kv: int) -> int:
+    """Query heads per kv head. The API page's ulysses_attention takes q with
+    Hq heads and k/v with Hkv heads; each kv head serves Hq / Hkv consecutive
+    query heads."""
+    if heads_kv < 1 or heads_q % heads_kv != 0:
+        raise ValueError(f"query heads ({heads_q}) must be a multiple of kv heads ({heads_kv})")
+    return heads_q // heads_kv
+
+
+def check_gqa_ranges(head_ranges, kv_head_ranges, group: int) -> None:
+    """Every rank must own the kv heads its query heads use (the head split must
+    keep groups whole on each rank, as a sharding divisible by the group size
+    does). Raises ValueError otherwise."""
+    for r, ((h0, h1), (k0, k1)) in enumerate(zip(head_ranges, kv_head_ranges, strict=True)):
+        for h in range(h0, h1):
+            if not k0 <= h // group < k1:
+                raise ValueError(f"rank {r}: query head {h} uses kv head {h // group}, outside its kv heads [{k0}, {k1})")

@@ -142,3 +142,44 @@ def test_default_scale():
     assert default_scale(128) == 1.0 / math.sqrt(128)
     q, k, v = (_rand((1, 7, 2, 16), s) for s in (61, 62, 63))
     np.testing.assert_array_equal(attention_bshd(q, k, v), attention_bshd(q, k, v, scale=0.25))
+
+
+# ---------------------------------------------------------------- grouped-query attention
+def test_gqa_matches_torch_sdpa_float64():
+    q, k, v = _rand((1, 37, 6, 16), 71), _rand((1, 37, 2, 16), 72), _rand((1, 37, 2, 16), 73)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).permute(0, 2, 1, 3), torch.from_numpy(k).permute(0, 2, 1, 3),
+        torch.from_numpy(v).permute(0, 2, 1, 3), enable_gqa=True).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(attention_bshd(q, k, v), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    q, k, v = _rand((2, 21, 8, 8), 74), _rand((2, 21, 2, 8), 75), _rand((2, 21, 2, 8), 76)
+    mha = attention_bshd(q, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2))
+    np.testing.assert_array_equal(attention_bshd(q, k, v), mha)
+
+
+@pytest.mark.parametrize("case", [(1, 37, 8, 4, 16, 4, 0), (2, 23, 12, 4, 8, 2, 1), (1, 19, 6, 6, 8, 3, 0),
+                                  (3, 16, 16, 8, 8, 4, 1)])
+def test_ulysses_gqa_equals_full_attention(case):
+    batch, tokens, hq, hkv, dim, world, prefix = case
+    tr, hr, kr = balanced_ranges(tokens, world), balanced_ranges(hq, world), balanced_ranges(hkv, world)
+    q = _rand((batch, prefix + tokens, hq, dim), 81)
+    k, v = _rand((batch, prefix + tokens, hkv, dim), 82), _rand((batch, prefix + tokens, hkv, dim), 83)
+    qs, ks, vs = (scatter_sequence(x, tr, prefix=prefix) for x in (q, k, v))
+    ref = scatter_sequence(attention_bshd(q, k, v), tr, prefix=prefix)
+    for n in (1, 2, 5):
+        out = ulysses_attention(qs, ks, vs, tr, hr, kv_head_ranges=kr, prefix=prefix, num_chunks=n)
+        for a, b in zip(out, ref):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_gqa_split_that_breaks_groups_is_rejected():
+    # 6 query heads over 4 ranks -> 2,2,1,1; 3 kv heads -> 1,1,1,0 is impossible
+    # (fewer kv heads than ranks); 12 q / 4 kv over 3 ranks -> q 4,4,4 with kv 2,1,1:
+    # rank 0's query heads 0..3 use kv heads 0,1 (owned), rank 1's 4..7 use 2,3 but owns only 2.
+    tr, hr, kr = balanced_ranges(9, 3), balanced_ranges(12, 3), balanced_ranges(4, 3)
+    x = [np.zeros((1, 3, 4, 2))] * 3
+    kv = [np.zeros((1, 3, b - a, 2)) for a, b in kr]
+    with pytest.raises(ValueError):
+        ulysses_attention(x, kv, kv, tr, hr, kv_head_ranges=kr)
