@@ -108,6 +108,23 @@ int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_ou
 int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads,
                     int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens);
 
+/*
+ * usp_plan_create_gqa -- as usp_plan_create, with grouped-query attention
+ * (API page, ulysses_attention: q is [seq/P, Hq, D], k/v are [seq/P, Hkv, D]).
+ * `heads` query heads and `heads_kv` k/v heads are each split by the balanced
+ * rule; query head h uses kv head h / (heads / heads_kv). Errors as
+ * usp_plan_create, plus USP_ERR_INVALID_ARG if heads is not a positive multiple
+ * of heads_kv or heads_kv < world, and USP_ERR_SHAPE if some rank's query heads
+ * use kv heads another rank owns (the API page's rule, both counts divisible by
+ * world, always satisfies this). usp_plan_create is this call with
+ * heads_kv = heads.
+ */
+int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                        int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens);
+
+/* Copies the plan's k/v head count and per-rank kv head ranges out; any output may be NULL. */
+int usp_plan_query_kv(const usp_plan* plan, int32_t* heads_kv, int32_t* kv_head_start, int32_t* kv_head_len);
+
 /* Releases the plan (synchronises its auxiliary stream first). NULL is ignored. */
 int usp_plan_destroy(usp_plan* plan);
 
@@ -158,6 +175,14 @@ int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* 
                             void* const* out, void* stream);
 
 /*
+ * usp_ulysses_seq_to_head_kv -- usp_ulysses_seq_to_head for k/v tensors under
+ * grouped-query attention: sequence shards [B, prefix+T_i, Hkv, D] become head
+ * shards [B, T', Hkv_r, D] over the plan's kv head ranges.
+ */
+int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
+                               void* stream);
+
+/*
  * usp_ulysses_head_to_seq -- "h3_blackwell_runtime/distributed.py",
  * SequenceParallelContext.heads_to_seq: head shards in[t*P + r] [B, T', H_r, D]
  * become sequence shards out[t*P + i] [B, prefix+T_i, H, D]:
@@ -174,21 +199,25 @@ int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* 
  * non-causal, no mask, over all T' tokens ("deepspeed/sequence/autosp_vit.py":
  * ViT attention is non-causal). scale <= 0 selects 1/sqrt(D). 16-bit types
  * accumulate in fp32 on the tensor cores (tcgen05) with P rounded to the
- * input type; fp32 runs in fp32 on the CUDA cores.
+ * input type; fp32 runs in fp32 on the CUDA cores. With grouped-query
+ * attention k_r/v_r are [B, T', Hkv_r, D] and global query head h uses global
+ * kv head h / (Hq / Hkv).
  */
 int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const void* const* k_heads,
                        const void* const* v_heads, void* const* o_heads, float scale, void* stream);
 
 /*
  * usp_ulysses_attention_workspace_size -- bytes of device workspace that
- * usp_ulysses_attention needs (the head-sharded q, k and v of all ranks).
+ * usp_ulysses_attention needs (the head-sharded q, k and v of all ranks:
+ * (Hq + 2 Hkv) * B * T' * D elements, each part 256-byte aligned).
  */
 int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunks, size_t* bytes);
 
 /*
  * usp_ulysses_attention -- API page, ulysses_attention, with the head-chunked
  * passes of "maxdiffusion PR #428": sequence shards q/k/v[i]
- * [B, prefix+T_i, H, D] in, sequence shards out[i] [B, prefix+T_i, H, D] out.
+ * [B, prefix+T_i, H, D] in (k/v with Hkv heads under grouped-query
+ * attention), sequence shards out[i] [B, prefix+T_i, H, D] out.
  * For each head chunk c (usp_head_chunk_ranges over G = max H_r, the same
  * local-head window on every rank, clipped to H_r): the seq->head exchange of
  * chunk c's heads of q, k and v runs on the plan's auxiliary stream; the

@@ -70,6 +70,14 @@ def test_head_chunks_match_oracle(usp):
     (dict(batch=1, seq_len=8, heads=300, head_dim=16, world=4), "USP_ERR_INVALID_ARG"),
     (dict(batch=1, seq_len=8, heads=4, head_dim=16, world=4, prefix=2), "USP_ERR_INVALID_ARG"),
     (dict(batch=1, seq_len=8, heads=4, head_dim=16, world=4, dtype=9), "USP_ERR_DTYPE"),
+    # grouped-query attention: kv heads must divide q heads, split over every rank
+    (dict(batch=1, seq_len=8, heads=6, head_dim=16, world=2, kv_heads=4), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=8, heads=8, head_dim=16, world=4, kv_heads=2), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=8, heads=8, head_dim=16, world=2, kv_heads=0), "USP_ERR_INVALID_ARG"),
+    # q 4,4,4 over kv 2,1,1: rank 1's query heads 4..7 need kv heads 2 and 3
+    (dict(batch=1, seq_len=9, heads=12, head_dim=16, world=3, kv_heads=4), "USP_ERR_SHAPE"),
+    # fewer kv heads than ranks
+    (dict(batch=1, seq_len=9, heads=6, head_dim=16, world=4, kv_heads=2), "USP_ERR_INVALID_ARG"),
 ])
 def test_plan_rejects_bad_arguments_before_any_device_work(usp, args, code):
     with pytest.raises(usp.UspError) as e:

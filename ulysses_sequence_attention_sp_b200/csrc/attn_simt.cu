@@ -36,15 +36,16 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
   const int row = blockIdx.x * kRows + threadIdx.x / kTPR;
   const bool row_ok = row < T;
 
-  const float* qb = static_cast<const float*>(L.in.q) + hm * L.in.stride_head + b * L.in.stride_batch;
-  const float* kb = static_cast<const float*>(L.in.k) + hm * L.in.stride_head + b * L.in.stride_batch;
-  const float* vb = static_cast<const float*>(L.in.v) + hm * L.in.stride_head + b * L.in.stride_batch;
+  const int hk = (L.in.q_head_base + hm) / L.in.kv_group - L.in.kv_head_base;  // kv head of this query head
+  const float* qb = static_cast<const float*>(L.in.q) + hm * L.in.qv.stride_head + b * L.in.qv.stride_batch;
+  const float* kb = static_cast<const float*>(L.in.k) + hk * L.in.kvv.stride_head + b * L.in.kvv.stride_batch;
+  const float* vb = static_cast<const float*>(L.in.v) + hk * L.in.kvv.stride_head + b * L.in.kvv.stride_batch;
 
   float q[DPT], acc[DPT];
 #pragma unroll
   for (int i = 0; i < DPT; ++i) {
     const int d = sub * DPT + i;
-    q[i] = (row_ok && d < D) ? qb[static_cast<int64_t>(row) * L.in.stride_token + d] * scale_log2 : 0.f;
+    q[i] = (row_ok && d < D) ? qb[static_cast<int64_t>(row) * L.in.qv.stride_token + d] * scale_log2 : 0.f;
     acc[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
     for (int idx = threadIdx.x; idx < kKT * DP; idx += kThreads) {
       const int r = idx / DP, d = idx - r * DP;
       const bool ok = (k0 + r < T) && d < D;
-      const int64_t off = static_cast<int64_t>(k0 + r) * L.in.stride_token + d;
+      const int64_t off = static_cast<int64_t>(k0 + r) * L.in.kvv.stride_token + d;
       sk[idx] = ok ? kb[off] : 0.f;
       sv[idx] = ok ? vb[off] : 0.f;
     }

@@ -10,6 +10,9 @@
 // the Ulysses block that is the sequence shard of the rank owning the row's
 // token (the head->seq exchange, fused).
 //
+// Grouped-query attention: query head h reads k/v head
+// (q_head_base + h) / kv_group - kv_head_base of the k/v views.
+//
 // One CTA computes one 128-row query tile of one (batch, head), walking the
 // keys in tiles of 256 (S = Q K^T is one M128 N256 MMA per 16 columns of D,
 // the shape that runs the tensor core at its full rate):
@@ -113,6 +116,7 @@ struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v;   // boxes: Q 128 rows, K 256 rows, V 128 rows
   AttnOut out;
   int32_t tokens, batch, n_heads, pad0;
+  int32_t kv_group, q_head_base, kv_head_base, pad1;  // k/v head of query head h: (q_head_base + h) / kv_group - kv_head_base
   float scale_log2;
   uint16_t heads[USP_MAX_HEADS];
 };
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int hi = blockIdx.y / p.batch;
   const int b = blockIdx.y - hi * p.batch;
   const int hm = p.heads[hi];
+  const int hk = (p.q_head_base + hm) / p.kv_group - p.kv_head_base;  // grouped-query attention
   const int T = p.tokens;
   const int ntiles = (T + kBN - 1) / kBN;
 #ifdef USP_TRACE
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           return false;
         mbar_arrive_expect_tx(&bars->k_full[st], C::KUNIT_BYTES);
         const int a = n % C::NATOM;
-        tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hm, (n / C::NATOM) * kBN, b);
+        tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hk, (n / C::NATOM) * kBN, b);
         return true;
       };
       auto load_v = [&](int m) -> bool {
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           return false;
         mbar_arrive_expect_tx(&bars->v_full[st], C::VHALF_BYTES);
         for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::VHALF_BYTES + a * C::VBLOCK_BYTES, a * C::ATOM, hm,
+          tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::VHALF_BYTES + a * C::VBLOCK_BYTES, a * C::ATOM, hk,
                       (m / 2) * kBN + (m % 2) * (kBN / 2), b);
         return true;
       };
@@ -511,14 +516,14 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-int make_map(CUtensorMap* map, const void* base, const AttnLaunch& L, int atom, int box_rows) {
+int make_map(CUtensorMap* map, const void* base, const AttnView& view, const AttnLaunch& L, int atom, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return set_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int e = 2;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(L.head_dim), static_cast<cuuint64_t>(L.in.head_extent),
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(L.head_dim), static_cast<cuuint64_t>(view.head_extent),
                         static_cast<cuuint64_t>(L.tokens), static_cast<cuuint64_t>(L.batch)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(L.in.stride_head * e), static_cast<cuuint64_t>(L.in.stride_token * e),
-                           static_cast<cuuint64_t>(L.in.stride_batch * e)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(view.stride_head * e), static_cast<cuuint64_t>(view.stride_token * e),
+                           static_cast<cuuint64_t>(view.stride_batch * e)};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(atom), 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUtensorMapSwizzle swz = atom == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -544,9 +549,12 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   TcParams p;
   memset(&p, 0, sizeof(p));
   int rc;
-  if ((rc = make_map(&p.tm_q, L.in.q, L, C::ATOM, kBM)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_k, L.in.k, L, C::ATOM, kBN)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_v, L.in.v, L, C::ATOM, kBN / 2)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_q, L.in.q, L.in.qv, L, C::ATOM, kBM)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_k, L.in.k, L.in.kvv, L, C::ATOM, kBN)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_v, L.in.v, L.in.kvv, L, C::ATOM, kBN / 2)) != USP_OK) return rc;
+  p.kv_group = L.in.kv_group;
+  p.q_head_base = L.in.q_head_base;
+  p.kv_head_base = L.in.kv_head_base;
   p.out = L.out;
   p.tokens = L.tokens;
   p.batch = L.batch;

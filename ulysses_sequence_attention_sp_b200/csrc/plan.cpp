@@ -119,8 +119,12 @@ void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) 
     }
 }
 
+// kv selects the k/v head geometry (Hkv heads split by kv_head_start) instead
+// of the query geometry.
 int seq_head_exchange(const usp_plan* plan, int dir, int32_t ntensors, const void* const* seq, void* const* heads,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool kv = false) {
+  const int32_t nheads = kv ? plan->heads_kv : plan->heads;
+  const int32_t* hstart = kv ? plan->kv_head_start : plan->head_start;
   usp::PermuteArgs a;
   memset(&a, 0, sizeof(a));
   const int64_t unit = static_cast<int64_t>(plan->head_dim) * plan->elem;
@@ -129,12 +133,12 @@ int seq_head_exchange(const usp_plan* plan, int dir, int32_t ntensors, const voi
   fill_seq_side(a, plan, plan->batch);
   a.n_head = plan->world;
   a.ntensors = ntensors;
-  a.heads = plan->heads;
+  a.heads = nheads;
   a.dv = static_cast<int32_t>(unit / vec);
   a.head_layout = 0;
   a.full_tokens = plan->tokens();
-  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = plan->head_start[r];
-  select_all_heads(a, plan->heads, plan->head_start, plan->world);
+  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = hstart[r];
+  select_all_heads(a, nheads, hstart, plan->world);
   for (int t = 0; t < ntensors; ++t)
     for (int r = 0; r < plan->world; ++r) {
       a.seq_ptr[t][r] = const_cast<void*>(seq[t * plan->world + r]);
@@ -200,6 +204,11 @@ int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_ou
 
 int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim, int32_t world,
                     int32_t dtype, int32_t prefix_tokens) {
+  return usp_plan_create_gqa(out, batch, seq_len, heads, heads, head_dim, world, dtype, prefix_tokens);
+}
+
+int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                        int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens) {
   if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (world < 1 || world > USP_MAX_WORLD)
@@ -231,6 +240,37 @@ int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t head
       }
       p->head_start[world] = heads;
       p->group_heads = p->head_len[0];
+    }
+  }
+  // Grouped-query attention: kv heads split the same way; every rank must own
+  // the kv heads its query heads use (query head h uses kv head h / group).
+  if (rc == USP_OK) {
+    if (heads_kv < 1 || heads % heads_kv != 0)
+      rc = usp::set_error(USP_ERR_INVALID_ARG, "query heads (%d) must be a positive multiple of kv heads (%d)", heads,
+                          heads_kv);
+  }
+  if (rc == USP_OK) {
+    int64_t ks[USP_MAX_WORLD], kl[USP_MAX_WORLD];
+    rc = balanced(heads_kv, world, ks, kl);
+    if (rc == USP_OK) {
+      p->heads_kv = heads_kv;
+      p->kv_group = heads / heads_kv;
+      for (int r = 0; r < world; ++r) {
+        p->kv_head_start[r] = static_cast<int32_t>(ks[r]);
+        p->kv_head_len[r] = static_cast<int32_t>(kl[r]);
+      }
+      p->kv_head_start[world] = heads_kv;
+      for (int r = 0; rc == USP_OK && r < world; ++r)
+        for (int h = p->head_start[r]; h < p->head_start[r + 1]; ++h) {
+          const int kvh = h / p->kv_group;
+          if (kvh < p->kv_head_start[r] || kvh >= p->kv_head_start[r + 1]) {
+            rc = usp::set_error(USP_ERR_SHAPE,
+                                "rank %d: query head %d uses kv head %d, outside its kv heads [%d, %d); choose "
+                                "head counts whose split keeps each group on one rank (e.g. both divisible by world)",
+                                r, h, kvh, p->kv_head_start[r], p->kv_head_start[r + 1]);
+            break;
+          }
+        }
     }
   }
   if (rc != USP_OK) {
@@ -269,6 +309,16 @@ int usp_plan_destroy(usp_plan* plan) {
   if (plan->ev_inputs) cudaEventDestroy(plan->ev_inputs);
   for (cudaEvent_t ev : plan->ev_chunk) cudaEventDestroy(ev);
   delete plan;
+  return USP_OK;
+}
+
+int usp_plan_query_kv(const usp_plan* plan, int32_t* heads_kv, int32_t* kv_head_start, int32_t* kv_head_len) {
+  if (int rc = check_plan(plan)) return rc;
+  if (heads_kv) *heads_kv = plan->heads_kv;
+  for (int r = 0; r < plan->world; ++r) {
+    if (kv_head_start) kv_head_start[r] = plan->kv_head_start[r];
+    if (kv_head_len) kv_head_len[r] = plan->kv_head_len[r];
+  }
   return USP_OK;
 }
 
@@ -389,6 +439,16 @@ int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* 
   return seq_head_exchange(plan, 0, ntensors, in, out, static_cast<cudaStream_t>(stream));
 }
 
+int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
+                               void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
+  if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  return seq_head_exchange(plan, 0, ntensors, in, out, static_cast<cudaStream_t>(stream), true);
+}
+
 int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
   if (int rc = check_plan(plan)) return rc;
@@ -434,7 +494,15 @@ int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const v
     usp::AttnLaunch L;
     memset(&L, 0, sizeof(L));
     const int64_t hr = plan->head_len[r];
-    L.in = {q_heads[r], k_heads[r], v_heads[r], D, hr * D, T * hr * D, hr};
+    const int64_t kr = plan->kv_head_len[r];
+    L.in.q = q_heads[r];
+    L.in.k = k_heads[r];
+    L.in.v = v_heads[r];
+    L.in.qv = {D, hr * D, T * hr * D, hr};
+    L.in.kvv = {D, kr * D, T * kr * D, kr};
+    L.in.kv_group = plan->kv_group;
+    L.in.q_head_base = plan->head_start[r];
+    L.in.kv_head_base = plan->kv_head_start[r];
     L.out.nseg = 1;
     L.out.prefix = 0;
     L.out.out_heads = static_cast<int32_t>(hr);
@@ -463,17 +531,40 @@ static int record_timing_event(cudaEvent_t ev, cudaStream_t s) {
   return usp::cuda_check(cudaEventRecordWithFlags(ev, s, flags), "cudaEventRecordWithFlags(timing)");
 }
 
-static size_t workspace_tensor_bytes(const usp_plan* plan) {
-  const size_t bytes = static_cast<size_t>(plan->batch) * plan->tokens() * plan->heads * plan->head_dim * plan->elem;
+// Bytes of one head-major workspace tensor with `heads` heads, 256-byte aligned.
+static size_t workspace_tensor_bytes(const usp_plan* plan, int32_t heads) {
+  const size_t bytes = static_cast<size_t>(plan->batch) * plan->tokens() * heads * plan->head_dim * plan->elem;
   return (bytes + 255) & ~size_t(255);
+}
+
+static size_t workspace_total_bytes(const usp_plan* plan) {
+  return workspace_tensor_bytes(plan, plan->heads) + 2 * workspace_tensor_bytes(plan, plan->heads_kv);
 }
 
 int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunks, size_t* bytes) {
   if (int rc = check_plan(plan)) return rc;
   if (!bytes) return usp::set_error(USP_ERR_INVALID_ARG, "bytes is NULL");
   if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive");
-  *bytes = 3 * workspace_tensor_bytes(plan);
+  *bytes = workspace_total_bytes(plan);
   return USP_OK;
+}
+
+// k/v heads packed with chunk window [lo, hi): on every rank, the kv heads whose
+// first query head lies in the window, so each kv head is packed exactly once
+// and before the first chunk that reads it.
+static void select_chunk_kv_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) {
+  a.nsel = 0;
+  const int g = p->kv_group;
+  for (int r = 0; r < p->world; ++r) {
+    if (lo >= p->head_len[r]) continue;
+    const int qa = p->head_start[r] + lo;
+    const int qb = p->head_start[r] + (hi < p->head_len[r] ? hi : p->head_len[r]);
+    for (int kvh = (qa + g - 1) / g; kvh * g < qb; ++kvh) {
+      a.sel_head[a.nsel] = static_cast<uint16_t>(kvh);
+      a.sel_rank[a.nsel] = static_cast<uint8_t>(r);
+      ++a.nsel;
+    }
+  }
 }
 
 int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void* const* k, const void* const* v,
@@ -488,54 +579,70 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
   if (!workspace) return usp::set_error(USP_ERR_INVALID_ARG, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return usp::set_error(USP_ERR_ALIGN, "workspace must be 256-byte aligned");
-  const size_t per = workspace_tensor_bytes(plan);
-  if (workspace_bytes < 3 * per)
-    return usp::set_error(USP_ERR_SHAPE, "workspace too small: %zu < %zu bytes", workspace_bytes, 3 * per);
+  const size_t need = workspace_total_bytes(plan);
+  if (workspace_bytes < need)
+    return usp::set_error(USP_ERR_SHAPE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   if (int rc = check_attention_shape(plan)) return rc;
   if (int rc = device_matches(plan)) return rc;
 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t T = plan->tokens(), D = plan->head_dim, B = plan->batch, H = plan->heads;
+  const int64_t T = plan->tokens(), D = plan->head_dim, B = plan->batch, H = plan->heads, HK = plan->heads_kv;
+  const bool gqa = plan->kv_group > 1;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* wq = ws;
-  void* wk = ws + per;
-  void* wv = ws + 2 * per;
+  void* wk = ws + workspace_tensor_bytes(plan, plan->heads);
+  void* wv = static_cast<uint8_t*>(wk) + workspace_tensor_bytes(plan, plan->heads_kv);
 
   // Head-chunk windows over the largest per-rank head group (rank 0's).
   int32_t nchunks = 0;
   int32_t lo[USP_MAX_HEADS], hi[USP_MAX_HEADS];
   usp_head_chunk_ranges(plan->group_heads, num_chunks, &nchunks, lo, hi);
 
-  // The seq->head exchange writes a head-major workspace [H][B][T'][D]: rank r's
-  // head shard is the contiguous block of its heads, so one 4-D view of the
-  // workspace covers every rank for the attention kernel.
-  usp::PermuteArgs a;
-  memset(&a, 0, sizeof(a));
+  // The seq->head exchange writes head-major workspaces [H][B][T'][D] (q) and
+  // [Hkv][B][T'][D] (k, v): rank r's head shard is the contiguous block of its
+  // heads, so one 4-D view of each workspace covers every rank for the
+  // attention kernel. Without grouped-query attention q, k and v move in one
+  // launch; with it, q and the k/v pair move in two (different head splits).
   const int64_t unit = D * plan->elem;
   const int vec = pick_vec(unit);
-  a.dir = 0;
-  fill_seq_side(a, plan, B);
-  a.n_head = plan->world;
-  a.ntensors = 3;
-  a.heads = static_cast<int32_t>(H);
-  a.dv = static_cast<int32_t>(unit / vec);
-  a.head_layout = 1;
-  a.full_tokens = T;
-  for (int r = 0; r <= plan->world; ++r) a.head_start[r] = plan->head_start[r];
-  const void* src[3] = {nullptr, nullptr, nullptr};
-  void* dst[3] = {wq, wk, wv};
+  auto pack_args = [&](usp::PermuteArgs& a, int32_t heads, const int32_t* hstart, int ntensors) {
+    memset(&a, 0, sizeof(a));
+    a.dir = 0;
+    fill_seq_side(a, plan, B);
+    a.n_head = plan->world;
+    a.ntensors = ntensors;
+    a.heads = heads;
+    a.dv = static_cast<int32_t>(unit / vec);
+    a.head_layout = 1;
+    a.full_tokens = T;
+    for (int r = 0; r <= plan->world; ++r) a.head_start[r] = hstart[r];
+  };
+  usp::PermuteArgs aq, akv;
+  pack_args(aq, static_cast<int32_t>(H), plan->head_start, gqa ? 1 : 3);
+  pack_args(akv, static_cast<int32_t>(HK), plan->kv_head_start, 2);
   for (int r = 0; r < plan->world; ++r) {
-    a.seq_ptr[0][r] = const_cast<void*>(q[r]);
-    a.seq_ptr[1][r] = const_cast<void*>(k[r]);
-    a.seq_ptr[2][r] = const_cast<void*>(v[r]);
-    const size_t off = static_cast<size_t>(plan->head_start[r]) * B * T * D * plan->elem;
-    for (int t = 0; t < 3; ++t) a.head_ptr[t][r] = static_cast<uint8_t*>(dst[t]) + off;
+    const size_t qoff = static_cast<size_t>(plan->head_start[r]) * B * T * D * plan->elem;
+    const size_t kvoff = static_cast<size_t>(plan->kv_head_start[r]) * B * T * D * plan->elem;
+    aq.seq_ptr[0][r] = const_cast<void*>(q[r]);
+    aq.head_ptr[0][r] = static_cast<uint8_t*>(wq) + qoff;
+    usp::PermuteArgs& kvargs = gqa ? akv : aq;
+    const int t0 = gqa ? 0 : 1;
+    kvargs.seq_ptr[t0][r] = const_cast<void*>(k[r]);
+    kvargs.seq_ptr[t0 + 1][r] = const_cast<void*>(v[r]);
+    kvargs.head_ptr[t0][r] = static_cast<uint8_t*>(wk) + kvoff;
+    kvargs.head_ptr[t0 + 1][r] = static_cast<uint8_t*>(wv) + kvoff;
   }
-  (void)src;
 
   usp::AttnLaunch L;
   memset(&L, 0, sizeof(L));
-  L.in = {wq, wk, wv, B * T * D, D, T * D, H};
+  L.in.q = wq;
+  L.in.k = wk;
+  L.in.v = wv;
+  L.in.qv = {B * T * D, D, T * D, H};
+  L.in.kvv = {B * T * D, D, T * D, HK};
+  L.in.kv_group = plan->kv_group;
+  L.in.q_head_base = 0;
+  L.in.kv_head_base = 0;
   L.out.nseg = plan->world;
   L.out.prefix = plan->prefix;
   L.out.out_heads = static_cast<int32_t>(H);
@@ -556,17 +663,20 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
     if (int rc = usp::cuda_check(cudaEventRecord(plan->ev_inputs, s), "cudaEventRecord")) return rc;
     if (int rc = usp::cuda_check(cudaStreamWaitEvent(plan->aux, plan->ev_inputs, 0), "cudaStreamWaitEvent")) return rc;
   }
+  const cudaStream_t ps = overlap ? plan->aux : s;
   for (int c = 0; c < nchunks; ++c) {
-    select_chunk_heads(a, plan, lo[c], hi[c]);
+    select_chunk_heads(aq, plan, lo[c], hi[c]);
+    if (int rc = usp::launch_permute(aq, vec, ps)) return rc;
+    if (gqa) {
+      select_chunk_kv_heads(akv, plan, lo[c], hi[c]);
+      if (int rc = usp::launch_permute(akv, vec, ps)) return rc;
+    }
     if (overlap) {
-      if (int rc = usp::launch_permute(a, vec, plan->aux)) return rc;
       if (int rc = usp::cuda_check(cudaEventRecord(plan->ev_chunk[c], plan->aux), "cudaEventRecord")) return rc;
       if (int rc = usp::cuda_check(cudaStreamWaitEvent(s, plan->ev_chunk[c], 0), "cudaStreamWaitEvent")) return rc;
-    } else {
-      if (int rc = usp::launch_permute(a, vec, s)) return rc;
     }
-    L.n_heads = a.nsel;
-    for (int i = 0; i < a.nsel; ++i) L.heads[i] = a.sel_head[i];
+    L.n_heads = aq.nsel;
+    for (int i = 0; i < aq.nsel; ++i) L.heads[i] = aq.sel_head[i];
     if (c == 0 && plan->t_start)
       if (int rc = record_timing_event(plan->t_start, s)) return rc;
     if (int rc = launch_attention(L, s)) return rc;

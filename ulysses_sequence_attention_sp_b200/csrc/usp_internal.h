@@ -23,6 +23,10 @@ struct usp_plan {
   int32_t head_start[USP_MAX_WORLD + 1] = {};
   int32_t head_len[USP_MAX_WORLD] = {};
   int32_t group_heads = 0;  // largest per-rank head count (rank 0's)
+  int32_t heads_kv = 0;     // k/v heads (== heads without grouped-query attention)
+  int32_t kv_group = 1;     // query heads per kv head
+  int32_t kv_head_start[USP_MAX_WORLD + 1] = {};
+  int32_t kv_head_len[USP_MAX_WORLD] = {};
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
@@ -84,16 +88,27 @@ struct AttnOut {
   void* seg_ptr[USP_MAX_WORLD];
 };
 
-// Inputs are 4-D views (d, head, token, batch) of q, k and v; the launch
-// processes every head coordinate in heads[0..n_heads) for every batch element.
-struct AttnInputs {
-  const void* q;
-  const void* k;
-  const void* v;
+// A 4-D view (d, head, token, batch) of one operand.
+struct AttnView {
   int64_t stride_head;   // elements
   int64_t stride_token;  // elements
   int64_t stride_batch;  // elements
   int64_t head_extent;   // head coordinates in the view
+};
+
+// The launch processes every q head coordinate in heads[0..n_heads) for every
+// batch element; q head coordinate h reads k/v head coordinate
+// (q_head_base + h) / kv_group - kv_head_base (grouped-query attention).
+struct AttnInputs {
+  const void* q;
+  const void* k;
+  const void* v;
+  AttnView qv;
+  AttnView kvv;
+  int32_t kv_group;
+  int32_t q_head_base;
+  int32_t kv_head_base;
+  int32_t pad0;
 };
 
 struct AttnLaunch {

@@ -7,7 +7,8 @@ round-to-nearest-even, and the oracle upcasts those exact bits.
 
 Recipe: ``numpy.random.default_rng(seed)``; q, k and v are drawn in that order
 from one stream with ``standard_normal(dtype=float32)`` times ``std``, in the
-full-sequence BSHD shape ``[batch, prefix + tokens, heads, head_dim]``.
+full-sequence BSHD shape ``[batch, prefix + tokens, heads, head_dim]`` (k and v
+with the workload's kv head count under grouped-query attention).
 Bit-pattern inputs for layout tests are uniform random 16- or 32-bit words.
 """
 
@@ -50,9 +51,10 @@ def make_qkv(w: Workload, seed: int | None = None):
     """Full-sequence q, k, v in storage form (uint16 bf16 bits, or float32)."""
     rng = np.random.default_rng(w.seed if seed is None else seed)
     shape = full_shape(w)
+    kv_shape = shape[:2] + (w.heads_kv,) + shape[3:]
     out = []
-    for _ in range(3):
-        x = rng.standard_normal(size=shape, dtype=np.float32)
+    for i in range(3):
+        x = rng.standard_normal(size=shape if i == 0 else kv_shape, dtype=np.float32)
         if w.std != 1.0:
             x *= np.float32(w.std)
         out.append(f32_to_bf16_bits(x) if w.dtype == "bf16" else x)

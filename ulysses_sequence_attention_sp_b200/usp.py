@@ -55,6 +55,12 @@ _SIGNATURES = {
     "usp_plan_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int64, ctypes.c_int64,
                                        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_int32]),
+    "usp_plan_create_gqa": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_int32]),
+    "usp_plan_query_kv": (ctypes.c_int, [ctypes.c_void_p, _c_i32p, _c_i32p, _c_i32p]),
+    "usp_ulysses_seq_to_head_kv": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, _c_vpp, _c_vpp,
+                                                  ctypes.c_void_p]),
     "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
     "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
@@ -155,14 +161,20 @@ def head_chunk_ranges(group_heads: int, num_chunks: int) -> list[tuple[int, int]
 
 # ------------------------------------------------------------------ plan
 class Plan:
-    """Token and head ownership of `world` virtual ranks on the current device."""
+    """Token and head ownership of `world` virtual ranks on the current device.
+
+    `kv_heads` (default: `heads`) gives k/v fewer heads than q (grouped-query
+    attention); query head h then uses kv head h // (heads // kv_heads)."""
 
     def __init__(self, batch: int, seq_len: int, heads: int, head_dim: int, world: int,
-                 dtype="bf16", prefix: int = 0):
+                 dtype="bf16", prefix: int = 0, kv_heads: int | None = None):
         code = _NAMES[dtype] if isinstance(dtype, str) else _DTYPES.get(dtype, dtype)
         handle = ctypes.c_void_p()
-        _check(_lib.usp_plan_create(ctypes.byref(handle), batch, seq_len, heads, head_dim, world, code, prefix))
+        kv_heads = heads if kv_heads is None else kv_heads
+        _check(_lib.usp_plan_create_gqa(ctypes.byref(handle), batch, seq_len, heads, kv_heads, head_dim, world,
+                                        code, prefix))
         self._h = handle
+        self.kv_heads = kv_heads
         self.batch, self.seq_len, self.heads, self.head_dim = batch, seq_len, heads, head_dim
         self.world, self.dtype_code, self.prefix = world, code, prefix
         self.torch_dtype = _TORCH[code]
@@ -171,6 +183,9 @@ class Plan:
         _check(_lib.usp_plan_query(self._h, ts, tl, hs, hl))
         self.token_ranges = tuple((ts[i], ts[i] + tl[i]) for i in range(world))
         self.head_ranges = tuple((hs[i], hs[i] + hl[i]) for i in range(world))
+        ks, kl = (ctypes.c_int32 * world)(), (ctypes.c_int32 * world)()
+        _check(_lib.usp_plan_query_kv(self._h, None, ks, kl))
+        self.kv_head_ranges = tuple((ks[i], ks[i] + kl[i]) for i in range(world))
 
     @property
     def handle(self):
@@ -192,6 +207,20 @@ class Plan:
     def head_shard_shape(self, r: int):
         h0, h1 = self.head_ranges[r]
         return (self.batch, self.tokens, h1 - h0, self.head_dim)
+
+    def kv_full_shape(self):
+        return (self.batch, self.tokens, self.kv_heads, self.head_dim)
+
+    def kv_seq_shard_shape(self, r: int):
+        t0, t1 = self.token_ranges[r]
+        return (self.batch, self.prefix + t1 - t0, self.kv_heads, self.head_dim)
+
+    def kv_head_shard_shape(self, r: int):
+        k0, k1 = self.kv_head_ranges[r]
+        return (self.batch, self.tokens, k1 - k0, self.head_dim)
+
+    def empty_kv_seq_shards(self, dtype=None, fill=None):
+        return [self._empty(self.kv_seq_shard_shape(r), dtype, fill) for r in range(self.world)]
 
     def empty_seq_shards(self, dtype=None, fill=None):
         return [self._empty(self.seq_shard_shape(r), dtype, fill) for r in range(self.world)]
@@ -251,22 +280,32 @@ def _check_tensors(plan: Plan, tensors, shapes, what: str) -> None:
 
 
 # --------------------------------------------------------- layout operations
+def _shard_shapes(plan: Plan, row_shape):
+    return [(plan.batch, plan.prefix + t1 - t0, *row_shape) for t0, t1 in plan.token_ranges]
+
+
 def scatter_sequence(plan: Plan, x_full, out=None, stream=None):
-    """API page, scatter_sequence: per-rank token windows of a replicated tensor."""
-    out = out if out is not None else [torch.empty(plan.seq_shard_shape(r), dtype=x_full.dtype, device=x_full.device)
-                                       for r in range(plan.world)]
-    _check_tensors(plan, [x_full], [plan.full_shape()], "x_full")
-    _check_tensors(plan, out, [plan.seq_shard_shape(r) for r in range(plan.world)], "x_shards")
-    _check(_lib.usp_scatter_sequence(plan.handle, x_full.data_ptr(), _ptrs(out), 0, 0, _stream(stream)))
+    """API page, scatter_sequence: per-rank token windows of a replicated tensor
+    [B, T', ...] (any row shape: q with H heads, k/v with Hkv heads, a hidden state)."""
+    row = tuple(x_full.shape[2:])
+    shapes = _shard_shapes(plan, row)
+    out = out if out is not None else [torch.empty(sh, dtype=x_full.dtype, device=x_full.device) for sh in shapes]
+    _check_tensors(plan, [x_full], [(plan.batch, plan.tokens, *row)], "x_full")
+    _check_tensors(plan, out, shapes, "x_shards")
+    row_bytes = x_full[0, 0].numel() * x_full.element_size()
+    _check(_lib.usp_scatter_sequence(plan.handle, x_full.data_ptr(), _ptrs(out), 0, row_bytes, _stream(stream)))
     return out
 
 
 def gather_sequence(plan: Plan, shards, out=None, stream=None):
     """API page, gather_sequence: the full tensor from the shards, in rank order."""
-    out = out if out is not None else torch.empty(plan.full_shape(), dtype=shards[0].dtype, device=shards[0].device)
-    _check_tensors(plan, shards, [plan.seq_shard_shape(r) for r in range(plan.world)], "x_shards")
-    _check_tensors(plan, [out], [plan.full_shape()], "x_full")
-    _check(_lib.usp_gather_sequence(plan.handle, _ptrs(shards), out.data_ptr(), 0, 0, _stream(stream)))
+    row = tuple(shards[0].shape[2:])
+    if out is None:
+        out = torch.empty((plan.batch, plan.tokens, *row), dtype=shards[0].dtype, device=shards[0].device)
+    _check_tensors(plan, shards, _shard_shapes(plan, row), "x_shards")
+    _check_tensors(plan, [out], [(plan.batch, plan.tokens, *row)], "x_full")
+    row_bytes = shards[0][0, 0].numel() * shards[0].element_size()
+    _check(_lib.usp_gather_sequence(plan.handle, _ptrs(shards), out.data_ptr(), 0, row_bytes, _stream(stream)))
     return out
 
 
@@ -290,18 +329,22 @@ def sp_head_gather(plan: Plan, head_shards, out=None, stream=None):
     return out
 
 
-def ulysses_seq_to_head(plan: Plan, tensors, out=None, stream=None):
+def ulysses_seq_to_head(plan: Plan, tensors, out=None, stream=None, kv: bool = False):
     """Ragged transport page, seq_to_heads: `tensors` is a list of 1..3 lists of
-    per-rank sequence shards (q, k, v); returns the matching per-rank head shards."""
+    per-rank sequence shards (q, k, v); returns the matching per-rank head shards.
+    kv=True moves k/v tensors over the plan's kv head split (grouped-query attention)."""
     n = len(tensors)
+    seq_shape = plan.kv_seq_shard_shape if kv else plan.seq_shard_shape
+    head_shape = plan.kv_head_shard_shape if kv else plan.head_shard_shape
     if out is None:
-        out = [[torch.empty(plan.head_shard_shape(r), dtype=tensors[0][0].dtype, device=tensors[0][0].device)
+        out = [[torch.empty(head_shape(r), dtype=tensors[0][0].dtype, device=tensors[0][0].device)
                 for r in range(plan.world)] for _ in range(n)]
     flat_in = [t for group in tensors for t in group]
     flat_out = [t for group in out for t in group]
-    _check_tensors(plan, flat_in, [plan.seq_shard_shape(r) for _ in range(n) for r in range(plan.world)], "in")
-    _check_tensors(plan, flat_out, [plan.head_shard_shape(r) for _ in range(n) for r in range(plan.world)], "out")
-    _check(_lib.usp_ulysses_seq_to_head(plan.handle, n, _ptrs(flat_in), _ptrs(flat_out), _stream(stream)))
+    _check_tensors(plan, flat_in, [seq_shape(r) for _ in range(n) for r in range(plan.world)], "in")
+    _check_tensors(plan, flat_out, [head_shape(r) for _ in range(n) for r in range(plan.world)], "out")
+    fn = _lib.usp_ulysses_seq_to_head_kv if kv else _lib.usp_ulysses_seq_to_head
+    _check(fn(plan.handle, n, _ptrs(flat_in), _ptrs(flat_out), _stream(stream)))
     return out
 
 
@@ -323,9 +366,11 @@ def ulysses_head_to_seq(plan: Plan, tensors, out=None, stream=None):
 def head_attention(plan: Plan, q_heads, k_heads, v_heads, out=None, scale: float = 0.0, stream=None):
     """run_attention on every rank's head shard (non-causal softmax attention)."""
     shapes = [plan.head_shard_shape(r) for r in range(plan.world)]
+    kv_shapes = [plan.kv_head_shard_shape(r) for r in range(plan.world)]
     out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
-    for name, ts in (("q_heads", q_heads), ("k_heads", k_heads), ("v_heads", v_heads), ("o_heads", out)):
-        _check_tensors(plan, ts, shapes, name)
+    for name, ts, sh in (("q_heads", q_heads, shapes), ("k_heads", k_heads, kv_shapes),
+                         ("v_heads", v_heads, kv_shapes), ("o_heads", out, shapes)):
+        _check_tensors(plan, ts, sh, name)
     _check(_lib.usp_head_attention(plan.handle, _ptrs(q_heads), _ptrs(k_heads), _ptrs(v_heads), _ptrs(out),
                                    float(scale), _stream(stream)))
     return out
@@ -336,9 +381,10 @@ def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chu
     """API page, ulysses_attention (with head-chunked passes): per-rank sequence
     shards of q, k, v in; per-rank sequence shards of the attention output out."""
     shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
+    kv_shapes = [plan.kv_seq_shard_shape(r) for r in range(plan.world)]
     out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
-    for name, ts in (("q", q), ("k", k), ("v", v), ("out", out)):
-        _check_tensors(plan, ts, shapes, name)
+    for name, ts, sh in (("q", q, shapes), ("k", k, kv_shapes), ("v", v, kv_shapes), ("out", out, shapes)):
+        _check_tensors(plan, ts, sh, name)
     need = plan.workspace_bytes(num_chunks)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
@@ -360,9 +406,10 @@ def ulysses_attention_noalloc(plan: Plan, q, k, v, out=None, scale: float = 0.0,
     all calls; calls that overlap on the GPU race). `out` must be given by such
     a caller; when it is None this helper allocates it with torch for convenience."""
     shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
+    kv_shapes = [plan.kv_seq_shard_shape(r) for r in range(plan.world)]
     out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
-    for name, ts in (("q", q), ("k", k), ("v", v), ("out", out)):
-        _check_tensors(plan, ts, shapes, name)
+    for name, ts, sh in (("q", q, shapes), ("k", k, kv_shapes), ("v", v, kv_shapes), ("out", out, shapes)):
+        _check_tensors(plan, ts, sh, name)
     _check(_lib.usp_ulysses_attention_noalloc(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
                                               num_chunks, _stream(stream)))
     return out

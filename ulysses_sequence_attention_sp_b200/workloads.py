@@ -22,6 +22,11 @@ class Workload:
     std: float
     seed: int
     num_chunks: tuple     # head-chunk counts the workload is run with
+    kv_heads: int = 0     # k/v heads (grouped-query attention); 0 means `heads`
+
+    @property
+    def heads_kv(self) -> int:
+        return self.kv_heads or self.heads
 
     @property
     def tokens(self) -> int:
