@@ -107,3 +107,44 @@ def test_attention_mistakes_are_caught():
         except ValueError:
             ok = False
         assert not ok, bad.__name__
+
+
+def test_row_collective_mistakes_are_caught():
+    """A reduce-scatter that forgets the destination's row offset (reads rows
+    0..T_r of every partial for every destination), or an all-gather that drops the zero-padding
+    strip (keeps max_rows per rank), fails the adjointness pin or the shape."""
+    from oracle.rows import all_gather_rows, reduce_scatter_rows
+
+    tr = balanced_ranges(10, 4)
+    rng = np.random.default_rng(3)
+    x = [rng.standard_normal((1, 10, 2)) for _ in range(4)]
+    y = [rng.standard_normal((1, b - a, 2)) for a, b in tr]
+
+    def wrong_rs(partials, token_ranges):
+        out = []
+        for r, (start, stop) in enumerate(token_ranges):
+            acc = np.zeros_like(partials[0][:, start:stop])
+            for p in partials:
+                acc = acc + p[:, 0:stop - start]  # mistake: destination offset dropped
+            out.append(acc)
+        return out
+
+    def adjoint_gap(rs, ag):
+        lhs = sum(float(np.sum(a * b)) for a, b in zip(rs(x, tr), y))
+        rhs = sum(float(np.sum(a * b)) for a, b in zip(x, ag(y, tr)))
+        return abs(lhs - rhs)
+
+    assert adjoint_gap(reduce_scatter_rows, all_gather_rows) < 1e-10
+    assert adjoint_gap(wrong_rs, all_gather_rows) > 1e-3
+
+    def wrong_ag(local, token_ranges):
+        m = max(b - a for a, b in token_ranges)
+        blocks = []
+        for v in local:
+            pad = np.zeros((v.shape[0], m, *v.shape[2:]))
+            pad[:, : v.shape[1]] = v
+            blocks.append(pad)
+        full = np.concatenate(blocks, axis=1)  # mistake: padding rows kept
+        return [full] * len(local)
+
+    assert wrong_ag(y, tr)[0].shape != all_gather_rows(y, tr)[0].shape
