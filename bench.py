@@ -441,6 +441,10 @@ def reshard_measurement(usp, torch, dev, pk, pk_kind):
         usp.scatter_sequence(plan, full, out=s)
     heads = [plan.empty_head_shards() for _ in range(3)]
     full2 = torch.empty_like(full)
+    # row collectives over the same split: P full replicas / P full partials
+    rows_local = [x.view(w.batch, x.shape[1], w.heads, w.head_dim) for x in seq[2]]
+    rows_full = [torch.empty_like(full) for _ in range(w.world)]
+    rows_out = [torch.empty_like(x) for x in rows_local]
     ops = {
         "seq_to_head_qkv": (lambda: usp.ulysses_seq_to_head(plan, seq, out=heads), 6 * S),
         "head_to_seq": (lambda: usp.ulysses_head_to_seq(plan, heads[:1], out=seq[:1]), 2 * S),
@@ -448,6 +452,8 @@ def reshard_measurement(usp, torch, dev, pk, pk_kind):
         "gather_sequence": (lambda: usp.gather_sequence(plan, seq[1], out=full2), 2 * S),
         "sp_head_slice": (lambda: usp.sp_head_slice(plan, full, out=heads[2]), 2 * S),
         "sp_head_gather": (lambda: usp.sp_head_gather(plan, heads[2], out=full2), 2 * S),
+        "all_gather_rows": (lambda: usp.all_gather_rows(plan, rows_local, out=rows_full), (1 + w.world) * S),
+        "reduce_scatter_rows": (lambda: usp.reduce_scatter_rows(plan, rows_full, out=rows_out), (w.world + 1) * S),
     }
     res = {}
     for name, (fn, nbytes) in ops.items():

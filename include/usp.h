@@ -193,6 +193,36 @@ int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* 
                             void* const* out, void* stream);
 
 /*
+ * usp_all_gather_rows -- "h3_blackwell_runtime/distributed.py",
+ * SequenceParallelContext.all_gather_rows: every rank receives all token rows,
+ * concatenated in rank order, with no padding in the result.
+ *   full_rows[r][b, t0_i + t, :] = local_rows[i][b, t, :]   for every r
+ * local_rows[i] is [outer, T_i, row] and full_rows[r] is [outer, T, row] (T =
+ * seq_len, the split tokens; the plan's prefix rows take no part), `row` =
+ * row_bytes bytes, a multiple of 2. outer = 0 and row_bytes = 0 mean B and
+ * H*D*elem. Caller-owned buffers, 16-byte aligned; outputs must not overlap
+ * inputs or each other. One kernel launch; reads S and writes P*S bytes.
+ * Errors: USP_ERR_INVALID_ARG (NULL pointer, bad sizes), USP_ERR_ALIGN,
+ * USP_ERR_CUDA.
+ */
+int usp_all_gather_rows(const usp_plan* plan, const void* const* local_rows, void* const* full_rows,
+                        int64_t outer, int64_t row_bytes, void* stream);
+
+/*
+ * usp_reduce_scatter_rows -- "h3_blackwell_runtime/distributed.py",
+ * SequenceParallelContext.reduce_scatter_rows: every rank holds a partial sum
+ * over all T token rows; rank r receives the sum over ranks of its own rows.
+ *   local_rows[r][b, t, :] = sum_{i=0..P-1} partial_full_rows[i][b, t0_r + t, :]
+ * partial_full_rows[i] is [outer, T, row] and local_rows[r] is [outer, T_r,
+ * row] of the plan's dtype; row_bytes as usp_all_gather_rows (a multiple of
+ * the element size). The sum runs in source-rank order in fp32 and is rounded
+ * once (round to nearest even) to the storage type. Buffers as above. One
+ * kernel launch; reads P*S and writes S bytes. Errors as usp_all_gather_rows.
+ */
+int usp_reduce_scatter_rows(const usp_plan* plan, const void* const* partial_full_rows, void* const* local_rows,
+                            int64_t outer, int64_t row_bytes, void* stream);
+
+/*
  * usp_head_attention -- API page, ulysses_attention's run_attention: the
  * unchanged single-device attention on every rank's head shard,
  *   o_r[b, :, h, :] = softmax(q_r[b, :, h, :] k_r[b, :, h, :]^T * scale) v_r[b, :, h, :]

@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(kThreads, 4) permute_kernel(const __grid_const
   }
 }
 
+}  // namespace
+
 int sm_count() {
   static int count = 0;
   if (count == 0) {
@@ -117,8 +119,6 @@ int sm_count() {
   }
   return count;
 }
-
-}  // namespace
 
 int launch_permute(const PermuteArgs& args, int vec_bytes, cudaStream_t stream) {
   PermuteArgs a = args;

@@ -429,6 +429,48 @@ int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, v
                            static_cast<cudaStream_t>(stream));
 }
 
+// Row collectives: the plan's token split, `outer` batches, rows of row_bytes.
+static int rows_collective(const usp_plan* plan, bool reduce, const void* const* src, void* const* dst,
+                           int64_t outer, int64_t row_bytes, void* stream) {
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_ptrs(src, plan->world, reduce ? "partial_full_rows" : "local_rows")) return rc;
+  if (int rc = check_ptrs(const_cast<const void* const*>(dst), plan->world, reduce ? "local_rows" : "full_rows"))
+    return rc;
+  if (int rc = device_matches(plan)) return rc;
+  if (outer == 0) outer = plan->batch;
+  if (row_bytes == 0) row_bytes = static_cast<int64_t>(plan->heads) * plan->head_dim * plan->elem;
+  if (outer < 1 || row_bytes < 1) return usp::set_error(USP_ERR_INVALID_ARG, "outer and row_bytes must be positive");
+  const int vec = pick_vec(row_bytes);
+  if (vec == 0) return usp::set_error(USP_ERR_INVALID_ARG, "row_bytes (%lld) must be even", (long long)row_bytes);
+  if (reduce && (row_bytes % plan->elem != 0 || vec < plan->elem))
+    return usp::set_error(USP_ERR_INVALID_ARG, "row_bytes (%lld) must be a multiple of the %d-byte element",
+                          (long long)row_bytes, plan->elem);
+  usp::RowsArgs a;
+  memset(&a, 0, sizeof(a));
+  a.world = plan->world;
+  a.outer = outer;
+  a.total_rows = plan->seq_len;
+  a.nv = row_bytes / vec;
+  for (int r = 0; r < plan->world; ++r) {
+    a.tok_start[r] = plan->tok_start[r];
+    a.tok_len[r] = plan->tok_len[r];
+    a.src[r] = src[r];
+    a.dst[r] = dst[r];
+  }
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return reduce ? usp::launch_reduce_scatter_rows(a, vec, plan->dtype, s) : usp::launch_all_gather_rows(a, vec, s);
+}
+
+int usp_all_gather_rows(const usp_plan* plan, const void* const* local_rows, void* const* full_rows, int64_t outer,
+                        int64_t row_bytes, void* stream) {
+  return rows_collective(plan, false, local_rows, full_rows, outer, row_bytes, stream);
+}
+
+int usp_reduce_scatter_rows(const usp_plan* plan, const void* const* partial_full_rows, void* const* local_rows,
+                            int64_t outer, int64_t row_bytes, void* stream) {
+  return rows_collective(plan, true, partial_full_rows, local_rows, outer, row_bytes, stream);
+}
+
 int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
   if (int rc = check_plan(plan)) return rc;

@@ -74,6 +74,30 @@ struct PermuteArgs {
 // vec_bytes in {16, 8, 4, 2}; dv counts vectors of that size.
 int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream);
 
+int sm_count();
+
+// ------------------------------------------------------- row collectives
+// Ragged row collectives over the plan's token split. Rank r's local buffer is
+// [outer][tok_len[r]][nv vectors]; a full buffer is [outer][total_rows][nv].
+// all_gather_rows: src = local buffers, dst = full buffers (one per rank).
+// reduce_scatter_rows: src = full partials, dst = local buffers.
+struct RowsArgs {
+  int32_t world;
+  int32_t pad0;
+  int64_t outer;
+  int64_t total_rows;
+  int64_t nv;  // vectors per row
+  int64_t tok_start[USP_MAX_WORLD];
+  int64_t tok_len[USP_MAX_WORLD];
+  int64_t seg_tiles[USP_MAX_WORLD];        // set by the launcher
+  int64_t tile_prefix[USP_MAX_WORLD + 1];  // set by the launcher
+  const void* src[USP_MAX_WORLD];
+  void* dst[USP_MAX_WORLD];
+};
+
+int launch_all_gather_rows(const RowsArgs& a, int vec_bytes, cudaStream_t stream);
+int launch_reduce_scatter_rows(const RowsArgs& a, int vec_bytes, int dtype, cudaStream_t stream);
+
 // -------------------------------------------------------------- attention
 // Where output rows go. Row t of (batch b, head g): rows t < prefix go to every
 // segment; other rows go to the segment s whose token range holds t - prefix.

@@ -61,6 +61,10 @@ _SIGNATURES = {
     "usp_plan_query_kv": (ctypes.c_int, [ctypes.c_void_p, _c_i32p, _c_i32p, _c_i32p]),
     "usp_ulysses_seq_to_head_kv": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, _c_vpp, _c_vpp,
                                                   ctypes.c_void_p]),
+    "usp_all_gather_rows": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_void_p]),
+    "usp_reduce_scatter_rows": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, ctypes.c_int64, ctypes.c_int64,
+                                               ctypes.c_void_p]),
     "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
     "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
@@ -359,6 +363,46 @@ def ulysses_head_to_seq(plan: Plan, tensors, out=None, stream=None):
     _check_tensors(plan, flat_in, [plan.head_shard_shape(r) for _ in range(n) for r in range(plan.world)], "in")
     _check_tensors(plan, flat_out, [plan.seq_shard_shape(r) for _ in range(n) for r in range(plan.world)], "out")
     _check(_lib.usp_ulysses_head_to_seq(plan.handle, n, _ptrs(flat_in), _ptrs(flat_out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------- row collectives
+def _row_shapes(plan: Plan, row_shape, full: bool):
+    if full:
+        return [(plan.batch, plan.seq_len, *row_shape)] * plan.world
+    return [(plan.batch, t1 - t0, *row_shape) for t0, t1 in plan.token_ranges]
+
+
+def all_gather_rows(plan: Plan, local_rows, out=None, stream=None):
+    """Ragged transport page, all_gather_rows: rank r's rows [B, T_r, ...] ->
+    every rank's full [B, T, ...] (T = the split tokens; no prefix rows)."""
+    row = tuple(local_rows[0].shape[2:])
+    if out is None:
+        out = [torch.empty(sh, dtype=local_rows[0].dtype, device=local_rows[0].device)
+               for sh in _row_shapes(plan, row, True)]
+    _check_tensors(plan, local_rows, _row_shapes(plan, row, False), "local_rows")
+    _check_tensors(plan, out, _row_shapes(plan, row, True), "full_rows")
+    row_bytes = local_rows[0][0, 0].numel() * local_rows[0].element_size()
+    _check(_lib.usp_all_gather_rows(plan.handle, _ptrs(local_rows), _ptrs(out), plan.batch, row_bytes,
+                                    _stream(stream)))
+    return out
+
+
+def reduce_scatter_rows(plan: Plan, partial_full_rows, out=None, stream=None):
+    """Ragged transport page, reduce_scatter_rows: every rank's partial
+    [B, T, ...] -> rank r's [B, T_r, ...] sum over ranks (fp32 accumulation)."""
+    row = tuple(partial_full_rows[0].shape[2:])
+    for t in partial_full_rows:
+        if t.dtype != plan.torch_dtype:
+            raise UspError(USP_ERR_DTYPE, f"partials are {t.dtype}, the plan sums {plan.torch_dtype}")
+    if out is None:
+        out = [torch.empty(sh, dtype=partial_full_rows[0].dtype, device=partial_full_rows[0].device)
+               for sh in _row_shapes(plan, row, False)]
+    _check_tensors(plan, partial_full_rows, _row_shapes(plan, row, True), "partial_full_rows")
+    _check_tensors(plan, out, _row_shapes(plan, row, False), "local_rows")
+    row_bytes = partial_full_rows[0][0, 0].numel() * partial_full_rows[0].element_size()
+    _check(_lib.usp_reduce_scatter_rows(plan.handle, _ptrs(partial_full_rows), _ptrs(out), plan.batch, row_bytes,
+                                        _stream(stream)))
     return out
 
 
