@@ -85,15 +85,19 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
+def recorded_traffic(kernel: str, algorithmic_bytes: float | None = None):
     """DRAM bytes per launch from the committed ncu summary, if the kernel
-    sources are unchanged since it was taken; else None."""
+    sources are unchanged since it was taken; else None. With
+    `algorithmic_bytes` (a launch of another size than the captured one), the
+    captured bytes are scaled by the ratio of algorithmic bytes."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         rec = json.load(f).get(kernel)
     if not rec or rec.get("source_hash") != source_hash(KERNEL_SOURCES[kernel]):
         return None
+    if algorithmic_bytes is not None and rec.get("algorithmic_bytes"):
+        return rec["bytes_per_launch"] * algorithmic_bytes / rec["algorithmic_bytes"]
     return rec.get("bytes_per_launch")
 
 
@@ -367,7 +371,8 @@ def run_ours(args, w, rank, world, local_rank):
         attn_launch_ms = attn_ms_max / n_launch_attn
         achieved = flop / n_launch_attn / (attn_launch_ms / 1e3) / 1e12
         peak_key = "bf16_tflops_sustained"
-        traffic = recorded_traffic("attention")
+        # algorithmic bytes of one launch: q, k, v read once and o written once
+        traffic = recorded_traffic("attention", 4 * w.tensor_bytes / n_launch_attn)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -474,7 +479,8 @@ def reshard_measurement(usp, torch, dev, pk, pk_kind):
     s2h = res["seq_to_head_qkv"]
     return {"workload": w.name, "ops": res, "peak_gbs": pk["hbm_gbs"], "peak_source": f"hbm_gbs ({pk_kind})",
             "roofline": {"bound": "hbm", "achieved": s2h["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": s2h["frac"], "traffic": recorded_traffic("permute"),
+                         "frac": s2h["frac"], "traffic": recorded_traffic("permute", 6 * S),
+                         "traffic_note": "ncu capture on the video workload's q/k/v pack, scaled by algorithmic bytes",
                          "kernel": "permute_kernel (seq_to_head of q, k, v)"}}
 
 
