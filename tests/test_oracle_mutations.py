@@ -148,3 +148,41 @@ def test_row_collective_mistakes_are_caught():
         return [full] * len(local)
 
     assert wrong_ag(y, tr)[0].shape != all_gather_rows(y, tr)[0].shape
+
+
+def test_ring_merge_mistakes_are_caught():
+    """A merge that averages the partials, or one that weights them by exp(lse)
+    without renormalising, fails the two-block pin; a cls key that every ring
+    step sees fails the full-attention pin."""
+    from oracle.attention import attention_bshd
+    from oracle.ring import block_attention, merge_partials
+
+    rng = np.random.default_rng(5)
+    q, k, v = rng.standard_normal((6, 8)) * 2, rng.standard_normal((30, 8)) * 2, rng.standard_normal((30, 8))
+    whole = block_attention(q, k, v, 0.7)
+    a, b = block_attention(q, k[:11], v[:11], 0.7), block_attention(q, k[11:], v[11:], 0.7)
+
+    def averaged(o_a, lse_a, o_b, lse_b):
+        return (o_a + o_b) / 2, np.logaddexp(lse_a, lse_b)
+
+    def unnormalised(o_a, lse_a, o_b, lse_b):
+        return o_a * np.exp(lse_a)[:, None] + o_b * np.exp(lse_b)[:, None], np.logaddexp(lse_a, lse_b)
+
+    assert np.allclose(merge_partials(*a, *b)[0], whole[0], rtol=1e-12, atol=1e-13)
+    for wrong in (averaged, unnormalised):
+        assert not np.allclose(wrong(*a, *b)[0], whole[0], rtol=1e-6, atol=1e-6)
+
+    # cls key in every block: attention over [cls, block] per step, merged
+    tokens, ring = 12, 3
+    x = [rng.standard_normal((1 + tokens, 4)) * 2 for _ in range(3)]
+    x[1][0] *= 3.0
+    qq, kk, vv = x
+    blocks = [(1 + 4 * g, 1 + 4 * (g + 1)) for g in range(ring)]
+    o = lse = None
+    for s0, s1 in blocks:
+        kb = np.concatenate([kk[:1], kk[s0:s1]])
+        vb = np.concatenate([vv[:1], vv[s0:s1]])
+        part = block_attention(qq, kb, vb, 0.5)
+        o, lse = part if o is None else merge_partials(o, lse, *part)
+    ref = attention_bshd(qq[None, :, None], kk[None, :, None], vv[None, :, None], scale=0.5)[0, :, 0]
+    assert not np.allclose(o, ref, rtol=1e-6, atol=1e-6)
