@@ -42,7 +42,8 @@ from ulysses_sequence_attention_sp_b200 import workloads as W  # noqa: E402
 from ulysses_sequence_attention_sp_b200.synth import make_qkv, storage_to_f64  # noqa: E402
 
 METRIC = "reshard GB/s and Ulysses-attention TFLOP/s on 1 B200, % of HBM/bf16 roofline"
-WORKLOADS = {"tiny": W.TINY, "reshard": W.RESHARD, "video": W.VIDEO, "vit": W.VIT, "chunked": W.CHUNKED}
+WORKLOADS = {"tiny": W.TINY, "reshard": W.RESHARD, "video": W.VIDEO, "vit": W.VIT, "chunked": W.CHUNKED,
+             "hybrid": W.HYBRID}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
@@ -246,7 +247,8 @@ def workload_config(w, num_chunks, n_gpus):
         "workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "prefix_tokens": w.prefix,
         "heads": w.heads, "head_dim": w.head_dim, "sp_virtual_ranks": w.world, "num_chunks": num_chunks,
         "global_batch": w.batch * n_gpus,
-        "parallelism": f"{n_gpus} independent replica(s), {w.world} virtual SP ranks each",
+        "parallelism": f"{n_gpus} independent replica(s), {w.world} virtual SP ranks each"
+                       + (f" (Ulysses {w.world // w.ring} x Ring {w.ring})" if w.ring > 1 else ""),
         "step": "scatter_sequence(q,k,v) -> ulysses_attention -> gather_sequence(out)",
         "l2": f"inputs larger than L2: {3 * w.tensor_bytes / 2**20:.0f} MiB of q/k/v per step"
         if 3 * w.tensor_bytes > 126 * 2**20 else "L2 flushed (512 MiB write) before every timed step",
@@ -264,7 +266,8 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.set_device(dev)
     n_chunks = args.num_chunks or w.num_chunks[0]
     pk, pk_kind = peaks()
-    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix)
+    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix, kv_heads=w.heads_kv,
+                    ring_size=w.ring)
     tdt = plan.torch_dtype
     storage = make_qkv(w, seed=w.seed + 7919 * rank)
 

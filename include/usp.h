@@ -125,6 +125,34 @@ int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t 
 /* Copies the plan's k/v head count and per-rank kv head ranges out; any output may be NULL. */
 int usp_plan_query_kv(const usp_plan* plan, int32_t* heads_kv, int32_t* kv_head_start, int32_t* kv_head_len);
 
+/*
+ * usp_plan_create_hybrid -- the Ulysses + Ring hybrid ("maxdiffusion PR #428:
+ * experimental two-phase (head-chunked) Ulysses all-to-all", which runs the
+ * head-chunked passes on plain Ulysses and on Ulysses+Ring). world =
+ * ulysses_size * ring_size virtual ranks split the tokens by the balanced
+ * rule. Ulysses group g is ranks g*ulysses_size .. (g+1)*ulysses_size - 1 and
+ * owns the contiguous token block of its members; inside a group the heads
+ * (and kv heads) are split over the ulysses_size members by the balanced
+ * rule, so rank r holds the heads of position u = r % ulysses_size. Ranks
+ * with the same u form a ring that passes k/v blocks; outputs of the blocks
+ * merge by their log-sum-exps. A prefix (cls) row is a key of block 0 only.
+ * With such a plan, usp_ulysses_attention(_lse, _noalloc) run the hybrid
+ * block, with the same arguments, workspace and chunking; scatter, gather and
+ * the row collectives work as for any plan; the per-rank head-shard calls
+ * (usp_ulysses_seq_to_head(_kv), usp_ulysses_head_to_seq, usp_sp_head_slice,
+ * usp_sp_head_gather, usp_head_attention) return USP_ERR_UNSUPPORTED.
+ * usp_plan_query reports rank r's head range as its position u's. Errors as
+ * usp_plan_create_gqa, with USP_ERR_INVALID_ARG if ulysses_size * ring_size is
+ * outside [1, USP_MAX_WORLD]. usp_plan_create_gqa is this call with
+ * ring_size = 1 and ulysses_size = world.
+ */
+int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                           int32_t head_dim, int32_t ulysses_size, int32_t ring_size, int32_t dtype,
+                           int32_t prefix_tokens);
+
+/* Copies the plan's Ulysses group size and ring size out (world and 1 for a plain plan); either may be NULL. */
+int usp_plan_query_hybrid(const usp_plan* plan, int32_t* ulysses_size, int32_t* ring_size);
+
 /* Releases the plan (synchronises its auxiliary stream first). NULL is ignored. */
 int usp_plan_destroy(usp_plan* plan);
 
@@ -263,6 +291,19 @@ int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunk
 int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void* const* k,
                           const void* const* v, void* const* out, float scale, int32_t num_chunks,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * usp_ulysses_attention_lse -- usp_ulysses_attention that also writes every
+ * output row's log-sum-exp (the row statistic a ring step or a backward pass
+ * merges with): lse[(h * B + b) * T' + t] = log sum_j exp(scale * q_t . k_j)
+ * over all T' keys, natural log, fp32, h the global query head and t the row
+ * in the full sequence (prefix rows first). lse is caller-owned device memory
+ * of H * B * T' floats, 4-byte aligned. Errors as usp_ulysses_attention, plus
+ * USP_ERR_INVALID_ARG for a NULL lse.
+ */
+int usp_ulysses_attention_lse(const usp_plan* plan, const void* const* q, const void* const* k,
+                              const void* const* v, void* const* out, float* lse, float scale, int32_t num_chunks,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * usp_ulysses_attention_noalloc -- the source pages have no counterpart; this

@@ -76,6 +76,12 @@ def test_head_chunks_match_oracle(usp):
     (dict(batch=1, seq_len=8, heads=8, head_dim=16, world=2, kv_heads=0), "USP_ERR_INVALID_ARG"),
     # q 4,4,4 over kv 2,1,1: rank 1's query heads 4..7 need kv heads 2 and 3
     (dict(batch=1, seq_len=9, heads=12, head_dim=16, world=3, kv_heads=4), "USP_ERR_SHAPE"),
+    # Ulysses + Ring hybrid: ring_size must divide world, world <= 32, heads >= ulysses ranks
+    (dict(batch=1, seq_len=64, heads=8, head_dim=16, world=8, ring_size=3), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=64, heads=32, head_dim=16, world=64, ring_size=2), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=64, heads=2, head_dim=16, world=8, ring_size=2), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=5, heads=4, head_dim=16, world=8, ring_size=2), "USP_ERR_INVALID_ARG"),
+    (dict(batch=1, seq_len=64, heads=4, head_dim=16, world=4, ring_size=0), "USP_ERR_INVALID_ARG"),
     # fewer kv heads than ranks
     (dict(batch=1, seq_len=9, heads=6, head_dim=16, world=4, kv_heads=2), "USP_ERR_INVALID_ARG"),
 ])

@@ -20,8 +20,16 @@ constexpr int kThreads = 128;
 constexpr int kRows = kThreads / kTPR;   // query rows per CTA
 constexpr int kKT = 32;                  // keys per smem tile
 
+struct SimtBlocks {
+  int32_t nq, nk;
+  int32_t q_start[USP_MAX_WORLD + 1];
+  int32_t q_tile_prefix[USP_MAX_WORLD + 1];
+  int32_t kv_start[USP_MAX_WORLD + 1];
+};
+
 template <int DPT>
-__global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_constant__ AttnLaunch L, float scale_log2) {
+__global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_constant__ AttnLaunch L,
+                                                             const __grid_constant__ SimtBlocks B, float scale_log2) {
   extern __shared__ float sh[];
   const int D = L.head_dim;
   const int DP = DPT * kTPR;  // padded head dim
@@ -33,8 +41,11 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
   const int hm = L.heads[hi];
   const int T = L.tokens;
   const int sub = threadIdx.x % kTPR;
-  const int row = blockIdx.x * kRows + threadIdx.x / kTPR;
-  const bool row_ok = row < T;
+  // query group of this CTA; its rows are [q_start[g], q_start[g+1])
+  int g = 0;
+  while (g + 1 < B.nq && static_cast<int>(blockIdx.x) >= B.q_tile_prefix[g + 1]) ++g;
+  const int row = B.q_start[g] + (static_cast<int>(blockIdx.x) - B.q_tile_prefix[g]) * kRows + threadIdx.x / kTPR;
+  const bool row_ok = row < B.q_start[g + 1];
 
   const int hk = (L.in.q_head_base + hm) / L.in.kv_group - L.in.kv_head_base;  // kv head of this query head
   const float* qb = static_cast<const float*>(L.in.q) + hm * L.in.qv.stride_head + b * L.in.qv.stride_batch;
@@ -50,17 +61,21 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
   }
   float m = -INFINITY, l = 0.f;
 
-  for (int k0 = 0; k0 < T; k0 += kKT) {
+  // key blocks in ring order g, g-1, ... (mod nk); each in smem tiles of kKT keys
+  int blk = g % B.nk;
+  for (int step = 0; step < B.nk; ++step, blk = blk == 0 ? B.nk - 1 : blk - 1)
+  for (int k0 = B.kv_start[blk]; k0 < B.kv_start[blk + 1]; k0 += kKT) {
+    const int kend = B.kv_start[blk + 1];
     __syncthreads();
     for (int idx = threadIdx.x; idx < kKT * DP; idx += kThreads) {
       const int r = idx / DP, d = idx - r * DP;
-      const bool ok = (k0 + r < T) && d < D;
+      const bool ok = (k0 + r < kend) && d < D;
       const int64_t off = static_cast<int64_t>(k0 + r) * L.in.kvv.stride_token + d;
       sk[idx] = ok ? kb[off] : 0.f;
       sv[idx] = ok ? vb[off] : 0.f;
     }
     __syncthreads();
-    const int nk = min(kKT, T - k0);
+    const int nk = min(kKT, kend - k0);
     float s[kKT];
     float mx = -INFINITY;
 #pragma unroll
@@ -88,6 +103,8 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
     m = m_new;
   }
   if (!row_ok) return;
+  if (L.lse != nullptr && sub == 0)  // sum_j exp(scale s_j) = 2^m * l
+    L.lse[(static_cast<int64_t>(hm) * L.batch + b) * T + row] = (m + log2f(l)) * 0.69314718055994531f;
 
   const AttnOut& out = L.out;
   int seg_lo, seg_hi;
@@ -125,8 +142,12 @@ int launch_dpt(const AttnLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(simt smem)");
   }
   const float scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
-  dim3 grid((L.tokens + kRows - 1) / kRows, L.batch * L.n_heads);
-  attn_simt_kernel<DPT><<<grid, kThreads, smem, stream>>>(L, scale_log2);
+  SimtBlocks B;
+  const int kv_tokens = L.kv_tokens > 0 ? L.kv_tokens : L.tokens;
+  if (!fill_blocks(L, kv_tokens, kRows, B.nq, B.nk, B.q_start, B.q_tile_prefix, B.kv_start))
+    return set_error(USP_ERR_INVALID_ARG, "internal: bad query-group or key-block table");
+  dim3 grid(B.q_tile_prefix[B.nq], L.batch * L.n_heads);
+  attn_simt_kernel<DPT><<<grid, kThreads, smem, stream>>>(L, B, scale_log2);
   count_launch();
   return cuda_check(cudaGetLastError(), "attention (fp32) launch");
 }

@@ -115,11 +115,38 @@ static_assert(sizeof(Bars) + 8 <= 5120, "barrier block outgrew its shared-memory
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v;   // boxes: Q 128 rows, K 256 rows, V 128 rows
   AttnOut out;
-  int32_t tokens, batch, n_heads, pad0;
+  float* lse;                     // optional [head][batch][tokens], natural log
+  int32_t tokens, batch, n_heads, kv_tokens;
   int32_t kv_group, q_head_base, kv_head_base, pad1;  // k/v head of query head h: (q_head_base + h) / kv_group - kv_head_base
   float scale_log2;
+  int32_t n_qgroups, n_kvblocks;
+  int32_t q_start[USP_MAX_WORLD + 1];
+  int32_t q_tile_prefix[USP_MAX_WORLD + 1];  // query tiles before group g
+  int32_t kv_start[USP_MAX_WORLD + 1];
   uint16_t heads[USP_MAX_HEADS];
 };
+
+// Key tile j of query group g: key blocks are taken in ring order g, g-1, ...
+// (mod n_kvblocks), each cut into tiles of kBN keys, the last one ragged.
+// Returns the tile's first key row and the number of its keys that belong to
+// its block (the rest are masked).
+struct KeyTile {
+  int key0;
+  int valid;
+};
+
+__device__ __forceinline__ KeyTile key_tile(const TcParams& p, int g, int j) {
+  const int nb = p.n_kvblocks;
+  int blk = g % nb;
+  for (int s = 0; s < nb; ++s) {
+    const int len = p.kv_start[blk + 1] - p.kv_start[blk];
+    const int nt = (len + kBN - 1) / kBN;
+    if (j < nt) return KeyTile{p.kv_start[blk] + j * kBN, len - j * kBN};
+    j -= nt;
+    blk = blk == 0 ? nb - 1 : blk - 1;
+  }
+  return KeyTile{0, 0};  // not reached for j < the group's tile count
+}
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return bf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
@@ -144,13 +171,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qtile = blockIdx.x;
   const int hi = blockIdx.y / p.batch;
   const int b = blockIdx.y - hi * p.batch;
   const int hm = p.heads[hi];
   const int hk = (p.q_head_base + hm) / p.kv_group - p.kv_head_base;  // grouped-query attention
   const int T = p.tokens;
-  const int ntiles = (T + kBN - 1) / kBN;
+  // Query group of this CTA; its tile's first row. Recomputed where needed
+  // rather than kept live through the key loop.
+  auto group_of_cta = [&]() {
+    int g = 0;
+    while (g + 1 < p.n_qgroups && static_cast<int>(blockIdx.x) >= p.q_tile_prefix[g + 1]) ++g;
+    return g;
+  };
+  auto first_row = [&](int g) { return p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_tile_prefix[g]) * kBM; };
+  int ntiles = 0;  // key tiles over all blocks
+  for (int k = 0; k < p.n_kvblocks; ++k) ntiles += (p.kv_start[k + 1] - p.kv_start[k] + kBN - 1) / kBN;
 #ifdef USP_TRACE
   const bool trace_cta = blockIdx.x == 7 && blockIdx.y == 0;
 #endif
@@ -191,12 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      const int g = group_of_cta();
+      const int q_row0 = first_row(g);
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int a = 0; a < C::NATOM; ++a)
-        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * kBM * C::ROWB, a * C::ATOM, hm, qtile * kBM, b);
+        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * kBM * C::ROWB, a * C::ATOM, hm, q_row0, b);
       // Unit n of K is atom block n % NATOM of key tile n / NATOM; half m of V is
       // keys [128(m%2), +128) of tile m / 2. Both are issued in the order the
       // tensor core consumes them: K of tile j+1 before V of tile j.
@@ -207,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           return false;
         mbar_arrive_expect_tx(&bars->k_full[st], C::KUNIT_BYTES);
         const int a = n % C::NATOM;
-        tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hk, (n / C::NATOM) * kBN, b);
+        const int key0 = key_tile(p, g, n / C::NATOM).key0;
+        tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hk, key0, b);
         return true;
       };
       auto load_v = [&](int m) -> bool {
@@ -216,9 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             !mbar_wait(&bars->v_empty[st], ((m / kVSlots) - 1) & 1, abort_flag, &g_attn_error, 11, kWaitLimitNs))
           return false;
         mbar_arrive_expect_tx(&bars->v_full[st], C::VHALF_BYTES);
+        const int key0 = key_tile(p, g, m / 2).key0 + (m % 2) * (kBN / 2);
         for (int a = 0; a < C::NATOM; ++a)
           tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::VHALF_BYTES + a * C::VBLOCK_BYTES, a * C::ATOM, hk,
-                      (m / 2) * kBN + (m % 2) * (kBN / 2), b);
+                      key0, b);
         return true;
       };
       int nk = 0, nv = 0;  // units issued
@@ -330,6 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float m = -INFINITY;  // running maximum, log2 domain (identical in the four parts)
     float l = 0.f;        // this part's running denominator
     bool ok = true;
+    // Keys of the current block from this tile on (blocks in ring order, as key_tile).
+    int kb_blk = group_of_cta() % p.n_kvblocks;
+    int kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
     for (int j = 0; j < ntiles; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, &g_attn_error, 30, kWaitLimitNs))) { ok = false; break; }
       if (threadIdx.x == 0) USP_TRACE_EV(5, j);
@@ -344,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_arrive(&bars->s_empty);
 
       float* s = reinterpret_cast<float*>(sr);
-      const int valid = T - j * kBN - part * kCols;  // valid columns of this part
+      const int valid = kb_left - part * kCols;  // valid columns of this part (kb_left >= kBN: all)
       if (valid < kCols) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
@@ -435,6 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(&bars->p_full);
       if (threadIdx.x == 0) USP_TRACE_EV(9, j);
+      kb_left -= kBN;
+      if (kb_left <= 0) {
+        kb_blk = kb_blk == 0 ? p.n_kvblocks - 1 : kb_blk - 1;
+        kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+      }
     }
     // Combine the four parts' denominators.
     if (ok) {
@@ -447,12 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort_flag, &g_attn_error, 33, kWaitLimitNs))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int t = qtile * kBM + row;
+      const int g = group_of_cta();
+      const int t = first_row(g) + row;
+      const bool row_ok = t < p.q_start[g + 1] && t < T;
+      if (p.lse != nullptr && part == 0 && row_ok)  // sum_j exp(scale s_j) = 2^m * l
+        p.lse[(static_cast<int64_t>(hm) * p.batch + b) * T + t] = (m + log2f(l)) * 0.69314718055994531f;
       const AttnOut& out = p.out;
       // Destination(s) of this row.
       int seg_lo = 0, seg_hi = 0;
       int64_t row_in_seg = 0;
-      if (t < T) {
+      if (row_ok) {
         if (t < out.prefix) {
           seg_lo = 0;
           seg_hi = out.nseg;
@@ -516,12 +567,13 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-int make_map(CUtensorMap* map, const void* base, const AttnView& view, const AttnLaunch& L, int atom, int box_rows) {
+int make_map(CUtensorMap* map, const void* base, const AttnView& view, const AttnLaunch& L, int64_t rows, int atom,
+             int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return set_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int e = 2;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(L.head_dim), static_cast<cuuint64_t>(view.head_extent),
-                        static_cast<cuuint64_t>(L.tokens), static_cast<cuuint64_t>(L.batch)};
+                        static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(L.batch)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(view.stride_head * e), static_cast<cuuint64_t>(view.stride_token * e),
                            static_cast<cuuint64_t>(view.stride_batch * e)};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(atom), 1, static_cast<cuuint32_t>(box_rows), 1};
@@ -549,9 +601,14 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   TcParams p;
   memset(&p, 0, sizeof(p));
   int rc;
-  if ((rc = make_map(&p.tm_q, L.in.q, L.in.qv, L, C::ATOM, kBM)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_k, L.in.k, L.in.kvv, L, C::ATOM, kBN)) != USP_OK) return rc;
-  if ((rc = make_map(&p.tm_v, L.in.v, L.in.kvv, L, C::ATOM, kBN / 2)) != USP_OK) return rc;
+  const int kv_tokens = L.kv_tokens > 0 ? L.kv_tokens : L.tokens;
+  if ((rc = make_map(&p.tm_q, L.in.q, L.in.qv, L, L.tokens, C::ATOM, kBM)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_k, L.in.k, L.in.kvv, L, kv_tokens, C::ATOM, kBN)) != USP_OK) return rc;
+  if ((rc = make_map(&p.tm_v, L.in.v, L.in.kvv, L, kv_tokens, C::ATOM, kBN / 2)) != USP_OK) return rc;
+  if (!fill_blocks(L, kv_tokens, kBM, p.n_qgroups, p.n_kvblocks, p.q_start, p.q_tile_prefix, p.kv_start))
+    return set_error(USP_ERR_INVALID_ARG, "internal: bad query-group or key-block table");
+  p.kv_tokens = kv_tokens;
+  p.lse = L.lse;
   p.kv_group = L.in.kv_group;
   p.q_head_base = L.in.q_head_base;
   p.kv_head_base = L.in.kv_head_base;
@@ -561,7 +618,7 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   p.n_heads = L.n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
   for (int i = 0; i < L.n_heads; ++i) p.heads[i] = L.heads[i];
-  dim3 grid((L.tokens + kBM - 1) / kBM, L.batch * L.n_heads);
+  dim3 grid(p.q_tile_prefix[p.n_qgroups], L.batch * L.n_heads);
   attn_tc_kernel<D, BF16><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   count_launch();
   return cuda_check(cudaGetLastError(), "attention (tcgen05) launch");

@@ -62,6 +62,14 @@ int check_ptrs(const void* const* ptrs, int n, const char* what) {
   return USP_OK;
 }
 
+// Per-rank head shards exist only in the plain block (one head range per rank).
+int check_flat(const usp_plan* plan, const char* what) {
+  if (plan->ring > 1)
+    return usp::set_error(USP_ERR_UNSUPPORTED, "%s: the plan is a Ulysses + Ring hybrid; its head shards are "
+                          "internal to usp_ulysses_attention", what);
+  return USP_OK;
+}
+
 int check_ptr(const void* p, const char* what) {
   if (!p) return usp::set_error(USP_ERR_INVALID_ARG, "%s is NULL", what);
   if (!aligned16(p)) return usp::set_error(USP_ERR_ALIGN, "%s is not 16-byte aligned", what);
@@ -111,7 +119,7 @@ void select_all_heads(usp::PermuteArgs& a, int heads, const int32_t* head_start,
 // Heads of local window [lo, hi) on every rank (ragged: clipped to H_r).
 void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) {
   a.nsel = 0;
-  for (int r = 0; r < p->world; ++r)
+  for (int r = 0; r < p->head_ranks; ++r)
     for (int h = lo; h < hi && h < p->head_len[r]; ++h) {
       a.sel_head[a.nsel] = static_cast<uint16_t>(p->head_start[r] + h);
       a.sel_rank[a.nsel] = static_cast<uint8_t>(r);
@@ -204,15 +212,24 @@ int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_ou
 
 int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim, int32_t world,
                     int32_t dtype, int32_t prefix_tokens) {
-  return usp_plan_create_gqa(out, batch, seq_len, heads, heads, head_dim, world, dtype, prefix_tokens);
+  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads, head_dim, world, 1, dtype, prefix_tokens);
 }
 
 int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
                         int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens) {
+  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads_kv, head_dim, world, 1, dtype, prefix_tokens);
+}
+
+int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                           int32_t head_dim, int32_t ulysses_size, int32_t ring_size, int32_t dtype,
+                           int32_t prefix_tokens) {
   if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
-  if (world < 1 || world > USP_MAX_WORLD)
-    return usp::set_error(USP_ERR_INVALID_ARG, "world must be in [1, %d] (got %d)", USP_MAX_WORLD, world);
+  if (ulysses_size < 1 || ring_size < 1 || static_cast<int64_t>(ulysses_size) * ring_size > USP_MAX_WORLD)
+    return usp::set_error(USP_ERR_INVALID_ARG, "ulysses_size * ring_size must be in [1, %d] (got %d x %d)",
+                          USP_MAX_WORLD, ulysses_size, ring_size);
+  const int32_t world = ulysses_size * ring_size;
+  const int32_t hr = ulysses_size;  // head ranks
   if (batch < 1) return usp::set_error(USP_ERR_INVALID_ARG, "batch must be positive");
   if (head_dim < 1) return usp::set_error(USP_ERR_INVALID_ARG, "head_dim must be positive");
   if (heads > USP_MAX_HEADS) return usp::set_error(USP_ERR_INVALID_ARG, "heads must be <= %d", USP_MAX_HEADS);
@@ -229,16 +246,18 @@ int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t 
   p->dtype = dtype;
   p->prefix = prefix_tokens;
   p->elem = e;
+  p->head_ranks = hr;
+  p->ring = ring_size;
   int rc = balanced(seq_len, world, p->tok_start, p->tok_len);
   if (rc == USP_OK) {
     int64_t hs[USP_MAX_WORLD], hl[USP_MAX_WORLD];
-    rc = balanced(heads, world, hs, hl);
+    rc = balanced(heads, hr, hs, hl);
     if (rc == USP_OK) {
-      for (int r = 0; r < world; ++r) {
+      for (int r = 0; r < hr; ++r) {
         p->head_start[r] = static_cast<int32_t>(hs[r]);
         p->head_len[r] = static_cast<int32_t>(hl[r]);
       }
-      p->head_start[world] = heads;
+      p->head_start[hr] = heads;
       p->group_heads = p->head_len[0];
     }
   }
@@ -251,16 +270,16 @@ int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t 
   }
   if (rc == USP_OK) {
     int64_t ks[USP_MAX_WORLD], kl[USP_MAX_WORLD];
-    rc = balanced(heads_kv, world, ks, kl);
+    rc = balanced(heads_kv, hr, ks, kl);
     if (rc == USP_OK) {
       p->heads_kv = heads_kv;
       p->kv_group = heads / heads_kv;
-      for (int r = 0; r < world; ++r) {
+      for (int r = 0; r < hr; ++r) {
         p->kv_head_start[r] = static_cast<int32_t>(ks[r]);
         p->kv_head_len[r] = static_cast<int32_t>(kl[r]);
       }
-      p->kv_head_start[world] = heads_kv;
-      for (int r = 0; rc == USP_OK && r < world; ++r)
+      p->kv_head_start[hr] = heads_kv;
+      for (int r = 0; rc == USP_OK && r < hr; ++r)
         for (int h = p->head_start[r]; h < p->head_start[r + 1]; ++h) {
           const int kvh = h / p->kv_group;
           if (kvh < p->kv_head_start[r] || kvh >= p->kv_head_start[r + 1]) {
@@ -316,9 +335,17 @@ int usp_plan_query_kv(const usp_plan* plan, int32_t* heads_kv, int32_t* kv_head_
   if (int rc = check_plan(plan)) return rc;
   if (heads_kv) *heads_kv = plan->heads_kv;
   for (int r = 0; r < plan->world; ++r) {
-    if (kv_head_start) kv_head_start[r] = plan->kv_head_start[r];
-    if (kv_head_len) kv_head_len[r] = plan->kv_head_len[r];
+    const int u = r % plan->head_ranks;  // rank r's position in its Ulysses group
+    if (kv_head_start) kv_head_start[r] = plan->kv_head_start[u];
+    if (kv_head_len) kv_head_len[r] = plan->kv_head_len[u];
   }
+  return USP_OK;
+}
+
+int usp_plan_query_hybrid(const usp_plan* plan, int32_t* ulysses_size, int32_t* ring_size) {
+  if (int rc = check_plan(plan)) return rc;
+  if (ulysses_size) *ulysses_size = plan->head_ranks;
+  if (ring_size) *ring_size = plan->ring;
   return USP_OK;
 }
 
@@ -328,8 +355,9 @@ int usp_plan_query(const usp_plan* plan, int64_t* tok_start, int64_t* tok_len, i
   for (int r = 0; r < plan->world; ++r) {
     if (tok_start) tok_start[r] = plan->tok_start[r];
     if (tok_len) tok_len[r] = plan->tok_len[r];
-    if (head_start) head_start[r] = plan->head_start[r];
-    if (head_len) head_len[r] = plan->head_len[r];
+    const int u = r % plan->head_ranks;  // rank r's position in its Ulysses group
+    if (head_start) head_start[r] = plan->head_start[u];
+    if (head_len) head_len[r] = plan->head_len[u];
   }
   return USP_OK;
 }
@@ -413,6 +441,7 @@ static int head_slice_gather(const usp_plan* plan, int dir, const void* full, vo
 int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards, int64_t rows,
                       void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_sp_head_slice")) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(x_head_shards), plan->world, "x_head_shards")) return rc;
   if (int rc = device_matches(plan)) return rc;
@@ -422,6 +451,7 @@ int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_h
 int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, void* x_full, int64_t rows,
                        void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_sp_head_gather")) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
   if (int rc = check_ptrs(x_head_shards, plan->world, "x_head_shards")) return rc;
   if (int rc = device_matches(plan)) return rc;
@@ -474,6 +504,7 @@ int usp_reduce_scatter_rows(const usp_plan* plan, const void* const* partial_ful
 int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_ulysses_seq_to_head")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
   if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
@@ -484,6 +515,7 @@ int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* 
 int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                                void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_ulysses_seq_to_head_kv")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
   if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
@@ -494,6 +526,7 @@ int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const voi
 int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_ulysses_head_to_seq")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
   if (int rc = check_ptrs(in, ntensors * plan->world, "in")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(out), ntensors * plan->world, "out")) return rc;
@@ -524,6 +557,7 @@ static float resolve_scale(const usp_plan* plan, float scale) {
 int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const void* const* k_heads,
                        const void* const* v_heads, void* const* o_heads, float scale, void* stream) {
   if (int rc = check_plan(plan)) return rc;
+  if (int rc = check_flat(plan, "usp_head_attention")) return rc;
   if (int rc = check_ptrs(q_heads, plan->world, "q_heads")) return rc;
   if (int rc = check_ptrs(k_heads, plan->world, "k_heads")) return rc;
   if (int rc = check_ptrs(v_heads, plan->world, "v_heads")) return rc;
@@ -597,7 +631,7 @@ int usp_ulysses_attention_workspace_size(const usp_plan* plan, int32_t num_chunk
 static void select_chunk_kv_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) {
   a.nsel = 0;
   const int g = p->kv_group;
-  for (int r = 0; r < p->world; ++r) {
+  for (int r = 0; r < p->head_ranks; ++r) {
     if (lo >= p->head_len[r]) continue;
     const int qa = p->head_start[r] + lo;
     const int qb = p->head_start[r] + (hi < p->head_len[r] ? hi : p->head_len[r]);
@@ -609,9 +643,27 @@ static void select_chunk_kv_heads(usp::PermuteArgs& a, const usp_plan* p, int lo
   }
 }
 
+static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, const void* const* k,
+                                  const void* const* v, void* const* out, float* lse, float scale, int32_t num_chunks,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void* const* k, const void* const* v,
                           void* const* out, float scale, int32_t num_chunks, void* workspace, size_t workspace_bytes,
                           void* stream) {
+  return ulysses_attention_impl(plan, q, k, v, out, nullptr, scale, num_chunks, workspace, workspace_bytes, stream);
+}
+
+int usp_ulysses_attention_lse(const usp_plan* plan, const void* const* q, const void* const* k, const void* const* v,
+                              void* const* out, float* lse, float scale, int32_t num_chunks, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!lse) return usp::set_error(USP_ERR_INVALID_ARG, "lse is NULL");
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return usp::set_error(USP_ERR_ALIGN, "lse must be 4-byte aligned");
+  return ulysses_attention_impl(plan, q, k, v, out, lse, scale, num_chunks, workspace, workspace_bytes, stream);
+}
+
+static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, const void* const* k,
+                                  const void* const* v, void* const* out, float* lse, float scale, int32_t num_chunks,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
   if (int rc = check_plan(plan)) return rc;
   if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive (got %d)", num_chunks);
   if (int rc = check_ptrs(q, plan->world, "q")) return rc;
@@ -651,26 +703,31 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
     memset(&a, 0, sizeof(a));
     a.dir = 0;
     fill_seq_side(a, plan, B);
-    a.n_head = plan->world;
+    a.n_head = plan->head_ranks;
     a.ntensors = ntensors;
     a.heads = heads;
     a.dv = static_cast<int32_t>(unit / vec);
     a.head_layout = 1;
     a.full_tokens = T;
-    for (int r = 0; r <= plan->world; ++r) a.head_start[r] = hstart[r];
+    for (int r = 0; r <= plan->head_ranks; ++r) a.head_start[r] = hstart[r];
   };
   usp::PermuteArgs aq, akv;
   pack_args(aq, static_cast<int32_t>(H), plan->head_start, gqa ? 1 : 3);
   pack_args(akv, static_cast<int32_t>(HK), plan->kv_head_start, 2);
+  usp::PermuteArgs& kvargs = gqa ? akv : aq;
+  const int t0 = gqa ? 0 : 1;
   for (int r = 0; r < plan->world; ++r) {
-    const size_t qoff = static_cast<size_t>(plan->head_start[r]) * B * T * D * plan->elem;
-    const size_t kvoff = static_cast<size_t>(plan->kv_head_start[r]) * B * T * D * plan->elem;
     aq.seq_ptr[0][r] = const_cast<void*>(q[r]);
-    aq.head_ptr[0][r] = static_cast<uint8_t*>(wq) + qoff;
-    usp::PermuteArgs& kvargs = gqa ? akv : aq;
-    const int t0 = gqa ? 0 : 1;
     kvargs.seq_ptr[t0][r] = const_cast<void*>(k[r]);
     kvargs.seq_ptr[t0 + 1][r] = const_cast<void*>(v[r]);
+  }
+  // Head-side buffers: one per head rank (every rank for the plain block; the
+  // Ulysses positions u of the hybrid, where rank (g, u) owns the token block g
+  // of head group u's buffer).
+  for (int r = 0; r < plan->head_ranks; ++r) {
+    const size_t qoff = static_cast<size_t>(plan->head_start[r]) * B * T * D * plan->elem;
+    const size_t kvoff = static_cast<size_t>(plan->kv_head_start[r]) * B * T * D * plan->elem;
+    aq.head_ptr[0][r] = static_cast<uint8_t*>(wq) + qoff;
     kvargs.head_ptr[t0][r] = static_cast<uint8_t*>(wk) + kvoff;
     kvargs.head_ptr[t0 + 1][r] = static_cast<uint8_t*>(wv) + kvoff;
   }
@@ -698,6 +755,17 @@ int usp_ulysses_attention(const usp_plan* plan, const void* const* q, const void
   L.head_dim = static_cast<int32_t>(D);
   L.dtype = plan->dtype;
   L.scale = resolve_scale(plan, scale);
+  L.lse = lse;
+  if (plan->ring > 1) {
+    // Ring: query group g = key block g = token block of Ulysses group g
+    // (block 0 also holds the prefix rows); group g takes the key blocks in
+    // ring order g, g-1, ... inside one kernel.
+    L.blocks.n_qgroups = L.blocks.n_kvblocks = plan->ring;
+    for (int g = 0; g < plan->ring; ++g)
+      L.blocks.q_start[g] = L.blocks.kv_start[g] =
+          g == 0 ? 0 : static_cast<int32_t>(plan->prefix + plan->tok_start[g * plan->head_ranks]);
+    L.blocks.q_start[plan->ring] = L.blocks.kv_start[plan->ring] = static_cast<int32_t>(T);
+  }
 
   const bool overlap = nchunks > 1;
   if (overlap) {

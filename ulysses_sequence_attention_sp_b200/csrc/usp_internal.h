@@ -27,6 +27,11 @@ struct usp_plan {
   int32_t kv_group = 1;     // query heads per kv head
   int32_t kv_head_start[USP_MAX_WORLD + 1] = {};
   int32_t kv_head_len[USP_MAX_WORLD] = {};
+  // Ulysses + Ring hybrid: heads are split over `head_ranks` = ulysses ranks
+  // (the head arrays above hold head_ranks entries); `ring` Ulysses groups of
+  // consecutive ranks. The plain block is head_ranks == world, ring == 1.
+  int32_t head_ranks = 0;
+  int32_t ring = 1;
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
@@ -135,10 +140,27 @@ struct AttnInputs {
   int32_t pad0;
 };
 
+// Query groups and key blocks of a launch (the Ulysses + Ring hybrid). Query
+// group g is rows [q_start[g], q_start[g+1]) of the q view's token axis; key
+// block k is rows [kv_start[k], kv_start[k+1]) of the k/v views' token axis.
+// Group g takes the key blocks in ring order g, g-1, ..., g-n_kvblocks+1
+// (mod n_kvblocks) and the online softmax carries its state across them.
+// n_qgroups = 0 means one group [0, tokens); n_kvblocks = 0 one block
+// [0, kv_tokens). Every group and block is non-empty.
+struct AttnBlocks {
+  int32_t n_qgroups;
+  int32_t n_kvblocks;
+  int32_t q_start[USP_MAX_WORLD + 1];
+  int32_t kv_start[USP_MAX_WORLD + 1];
+};
+
 struct AttnLaunch {
   AttnInputs in;
   AttnOut out;
-  int32_t tokens;  // T' (keys and queries per head)
+  AttnBlocks blocks;
+  float* lse;         // optional: [q head coordinate][batch][tokens] fp32, log-sum-exp (natural log) of the scaled scores
+  int32_t kv_tokens;  // rows of the k/v views (0: tokens)
+  int32_t tokens;  // T' (queries per head; keys too unless kv_tokens is set)
   int32_t batch;
   int32_t n_heads;
   int32_t head_dim;
@@ -146,6 +168,28 @@ struct AttnLaunch {
   float scale;
   uint16_t heads[USP_MAX_HEADS];
 };
+
+// Resolves the launch's AttnBlocks (defaults: one group, one block) into
+// explicit tables, with q_tile_prefix[g] = query tiles of `rows_per_tile` rows
+// before group g. Returns false if a table is not increasing from 0 <= start
+// to an end within the token counts.
+inline bool fill_blocks(const AttnLaunch& L, int kv_tokens, int rows_per_tile, int32_t& nq, int32_t& nk,
+                        int32_t* q_start, int32_t* q_tile_prefix, int32_t* kv_start) {
+  nq = L.blocks.n_qgroups > 0 ? L.blocks.n_qgroups : 1;
+  nk = L.blocks.n_kvblocks > 0 ? L.blocks.n_kvblocks : 1;
+  if (nq > USP_MAX_WORLD || nk > USP_MAX_WORLD) return false;
+  for (int i = 0; i <= nq; ++i) q_start[i] = L.blocks.n_qgroups > 0 ? L.blocks.q_start[i] : (i ? L.tokens : 0);
+  for (int i = 0; i <= nk; ++i) kv_start[i] = L.blocks.n_kvblocks > 0 ? L.blocks.kv_start[i] : (i ? kv_tokens : 0);
+  if (q_start[0] < 0 || q_start[nq] > L.tokens || kv_start[0] < 0 || kv_start[nk] > kv_tokens) return false;
+  q_tile_prefix[0] = 0;
+  for (int g = 0; g < nq; ++g) {
+    if (q_start[g + 1] <= q_start[g]) return false;
+    q_tile_prefix[g + 1] = q_tile_prefix[g] + (q_start[g + 1] - q_start[g] + rows_per_tile - 1) / rows_per_tile;
+  }
+  for (int k = 0; k < nk; ++k)
+    if (kv_start[k + 1] <= kv_start[k]) return false;
+  return true;
+}
 
 bool attention_tc_supported(int dtype, int head_dim);
 int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream);

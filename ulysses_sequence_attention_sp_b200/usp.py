@@ -65,6 +65,13 @@ _SIGNATURES = {
                                            ctypes.c_void_p]),
     "usp_reduce_scatter_rows": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, ctypes.c_int64, ctypes.c_int64,
                                                ctypes.c_void_p]),
+    "usp_plan_create_hybrid": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
+    "usp_plan_query_hybrid": (ctypes.c_int, [ctypes.c_void_p, _c_i32p, _c_i32p]),
+    "usp_ulysses_attention_lse": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_void_p,
+                                                 ctypes.c_float, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]),
     "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
     "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
@@ -168,17 +175,25 @@ class Plan:
     """Token and head ownership of `world` virtual ranks on the current device.
 
     `kv_heads` (default: `heads`) gives k/v fewer heads than q (grouped-query
-    attention); query head h then uses kv head h // (heads // kv_heads)."""
+    attention); query head h then uses kv head h // (heads // kv_heads).
+    `ring_size` > 1 makes a Ulysses + Ring hybrid: the `world` ranks form
+    ring_size Ulysses groups of world // ring_size consecutive ranks; heads are
+    split inside a group and k/v blocks travel around the ring of ranks that
+    hold the same heads."""
 
     def __init__(self, batch: int, seq_len: int, heads: int, head_dim: int, world: int,
-                 dtype="bf16", prefix: int = 0, kv_heads: int | None = None):
+                 dtype="bf16", prefix: int = 0, kv_heads: int | None = None, ring_size: int = 1):
         code = _NAMES[dtype] if isinstance(dtype, str) else _DTYPES.get(dtype, dtype)
         handle = ctypes.c_void_p()
         kv_heads = heads if kv_heads is None else kv_heads
-        _check(_lib.usp_plan_create_gqa(ctypes.byref(handle), batch, seq_len, heads, kv_heads, head_dim, world,
-                                        code, prefix))
+        if ring_size < 1 or world % ring_size != 0:
+            raise UspError(USP_ERR_INVALID_ARG, f"ring_size {ring_size} must divide world {world}")
+        _check(_lib.usp_plan_create_hybrid(ctypes.byref(handle), batch, seq_len, heads, kv_heads, head_dim,
+                                           world // ring_size, ring_size, code, prefix))
         self._h = handle
         self.kv_heads = kv_heads
+        self.ulysses_size = world // ring_size
+        self.ring_size = ring_size
         self.batch, self.seq_len, self.heads, self.head_dim = batch, seq_len, heads, head_dim
         self.world, self.dtype_code, self.prefix = world, code, prefix
         self.torch_dtype = _TORCH[code]
@@ -421,9 +436,11 @@ def head_attention(plan: Plan, q_heads, k_heads, v_heads, out=None, scale: float
 
 
 def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chunks: int = 1,
-                      workspace=None, stream=None):
+                      workspace=None, stream=None, lse=None):
     """API page, ulysses_attention (with head-chunked passes): per-rank sequence
-    shards of q, k, v in; per-rank sequence shards of the attention output out."""
+    shards of q, k, v in; per-rank sequence shards of the attention output out.
+    A Ulysses + Ring plan runs the hybrid block. `lse` (a float32 CUDA tensor
+    [H, B, T']) also receives every row's log-sum-exp."""
     shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
     kv_shapes = [plan.kv_seq_shard_shape(r) for r in range(plan.world)]
     out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
@@ -434,9 +451,17 @@ def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chu
         workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
     if workspace.numel() * workspace.element_size() < need:
         raise UspError(USP_ERR_SHAPE, f"workspace needs {need} bytes")
-    _check(_lib.usp_ulysses_attention(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
-                                      num_chunks, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                      _stream(stream)))
+    nbytes = workspace.numel() * workspace.element_size()
+    if lse is None:
+        _check(_lib.usp_ulysses_attention(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
+                                          num_chunks, workspace.data_ptr(), nbytes, _stream(stream)))
+        return out
+    if (not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous()
+            or tuple(lse.shape) != (plan.heads, plan.batch, plan.tokens)):
+        raise UspError(USP_ERR_SHAPE, f"lse must be a contiguous float32 CUDA tensor of shape "
+                                      f"{(plan.heads, plan.batch, plan.tokens)}")
+    _check(_lib.usp_ulysses_attention_lse(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), lse.data_ptr(),
+                                          float(scale), num_chunks, workspace.data_ptr(), nbytes, _stream(stream)))
     return out
 
 

@@ -23,6 +23,7 @@ class Workload:
     seed: int
     num_chunks: tuple     # head-chunk counts the workload is run with
     kv_heads: int = 0     # k/v heads (grouped-query attention); 0 means `heads`
+    ring: int = 1         # Ulysses + Ring hybrid: ring size (world // ring ranks per Ulysses group)
 
     @property
     def heads_kv(self) -> int:
@@ -52,5 +53,9 @@ VIDEO = Workload("video-T75600-H24-D128-P7-bf16", 1, 75600, 0, 24, 128, 7, "bf16
 VIT = Workload("vit-B16-cls1+576-H16-D80-P4-bf16", 16, 576, 1, 16, 80, 4, "bf16", 0.5, 1004, (1,))
 CHUNKED = Workload("chunked-T16384-H40-D128-P8-bf16", 1, 16384, 0, 40, 128, 8, "bf16", 1.0, 1005, (3, 1))
 
-ALL = (TINY, RESHARD, VIDEO, VIT, CHUNKED)
+# The video latent on 8 ranks as a Ulysses + Ring hybrid: 2 groups of 4 (6 heads per rank), 2-step ring.
+HYBRID = Workload("hybrid-video-T75600-H24-D128-U4xR2-bf16", 1, 75600, 0, 24, 128, 8, "bf16", 1.0, 1006, (1,),
+                  ring=2)
+
+ALL = (TINY, RESHARD, VIDEO, VIT, CHUNKED, HYBRID)
 BY_NAME = {w.name: w for w in ALL}
