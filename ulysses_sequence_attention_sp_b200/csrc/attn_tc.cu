@@ -13,6 +13,14 @@
 // Grouped-query attention: query head h reads k/v head
 // (q_head_base + h) / kv_group - kv_head_base of the k/v views.
 //
+// Ulysses + Ring hybrid (the RING instantiation): query rows come in groups
+// and keys in blocks; a CTA's query tile lies in one group g, and it takes
+// the key blocks in ring order g, g-1, ... (its own block first), each cut
+// into 256-key tiles with the block's ragged last tile masked. The online
+// softmax state (row maximum m, denominator l, O) carries across blocks: it is
+// the ring's log-sum-exp merge, done one tile at a time. Optionally every
+// row's log-sum-exp, (m + log2 l) ln 2, is written out.
+//
 // One CTA computes one 128-row query tile of one (batch, head), walking the
 // keys in tiles of 256 (S = Q K^T is one M128 N256 MMA per 16 columns of D,
 // the shape that runs the tensor core at its full rate):
@@ -115,13 +123,13 @@ static_assert(sizeof(Bars) + 8 <= 5120, "barrier block outgrew its shared-memory
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v;   // boxes: Q 128 rows, K 256 rows, V 128 rows
   AttnOut out;
-  float* lse;                     // optional [head][batch][tokens], natural log
+  float* lse;
   int32_t tokens, batch, n_heads, kv_tokens;
   int32_t kv_group, q_head_base, kv_head_base, pad1;  // k/v head of query head h: (q_head_base + h) / kv_group - kv_head_base
   float scale_log2;
   int32_t n_qgroups, n_kvblocks;
   int32_t q_start[USP_MAX_WORLD + 1];
-  int32_t q_tile_prefix[USP_MAX_WORLD + 1];  // query tiles before group g
+  int32_t q_tile_prefix[USP_MAX_WORLD + 1];
   int32_t kv_start[USP_MAX_WORLD + 1];
   uint16_t heads[USP_MAX_HEADS];
 };
@@ -158,7 +166,7 @@ __device__ __forceinline__ float2 unpack2(uint32_t w, bool bf16) {
   return __half22float2(h);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool RING>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -171,21 +179,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int qtile = blockIdx.x;
   const int hi = blockIdx.y / p.batch;
   const int b = blockIdx.y - hi * p.batch;
   const int hm = p.heads[hi];
   const int hk = (p.q_head_base + hm) / p.kv_group - p.kv_head_base;  // grouped-query attention
-  const int T = p.tokens;
-  // Query group of this CTA; its tile's first row. Recomputed where needed
-  // rather than kept live through the key loop.
+  const int T = p.tokens;  // query rows; the plain kernel also takes them as keys
   auto group_of_cta = [&]() {
     int g = 0;
-    while (g + 1 < p.n_qgroups && static_cast<int>(blockIdx.x) >= p.q_tile_prefix[g + 1]) ++g;
+    if constexpr (RING)
+      while (g + 1 < p.n_qgroups && static_cast<int>(blockIdx.x) >= p.q_tile_prefix[g + 1]) ++g;
     return g;
   };
-  auto first_row = [&](int g) { return p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_tile_prefix[g]) * kBM; };
-  int ntiles = 0;  // key tiles over all blocks
-  for (int k = 0; k < p.n_kvblocks; ++k) ntiles += (p.kv_start[k + 1] - p.kv_start[k] + kBN - 1) / kBN;
+  auto first_row = [&](int g) {
+    if constexpr (RING) return p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_tile_prefix[g]) * kBM;
+    return static_cast<int>(blockIdx.x) * kBM;
+  };
+  const int ntiles = [&]() {  // key tiles over all blocks
+    if constexpr (RING) {
+      int n = 0;
+      for (int k = 0; k < p.n_kvblocks; ++k) n += (p.kv_start[k + 1] - p.kv_start[k] + kBN - 1) / kBN;
+      return n;
+    }
+    return (T + kBN - 1) / kBN;
+  }();
 #ifdef USP_TRACE
   const bool trace_cta = blockIdx.x == 7 && blockIdx.y == 0;
 #endif
@@ -226,14 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int g = group_of_cta();
-      const int q_row0 = first_row(g);
+      int g = 0;
+      if constexpr (RING) g = group_of_cta();
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int a = 0; a < C::NATOM; ++a)
-        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * kBM * C::ROWB, a * C::ATOM, hm, q_row0, b);
+        tma_load_4d(&p.tm_q, &bars->q_full, sQ + a * kBM * C::ROWB, a * C::ATOM, hm, RING ? first_row(g) : qtile * kBM,
+                    b);
       // Unit n of K is atom block n % NATOM of key tile n / NATOM; half m of V is
       // keys [128(m%2), +128) of tile m / 2. Both are issued in the order the
       // tensor core consumes them: K of tile j+1 before V of tile j.
@@ -244,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           return false;
         mbar_arrive_expect_tx(&bars->k_full[st], C::KUNIT_BYTES);
         const int a = n % C::NATOM;
-        const int key0 = key_tile(p, g, n / C::NATOM).key0;
+        const int key0 = RING ? key_tile(p, g, n / C::NATOM).key0 : (n / C::NATOM) * kBN;
         tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::KUNIT_BYTES, a * C::ATOM, hk, key0, b);
         return true;
       };
@@ -254,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             !mbar_wait(&bars->v_empty[st], ((m / kVSlots) - 1) & 1, abort_flag, &g_attn_error, 11, kWaitLimitNs))
           return false;
         mbar_arrive_expect_tx(&bars->v_full[st], C::VHALF_BYTES);
-        const int key0 = key_tile(p, g, m / 2).key0 + (m % 2) * (kBN / 2);
+        const int key0 = (RING ? key_tile(p, g, m / 2).key0 : (m / 2) * kBN) + (m % 2) * (kBN / 2);
         for (int a = 0; a < C::NATOM; ++a)
           tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::VHALF_BYTES + a * C::VBLOCK_BYTES, a * C::ATOM, hk,
                       key0, b);
@@ -366,12 +384,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float* xch = bars->xch;                          // [parity][part][row]
     uint64_t* xbar = &bars->xbar[quarter];
     const float sl2 = p.scale_log2;
+    int kb_blk = 0, kb_left = 0;
+    if constexpr (RING) {
+      kb_blk = group_of_cta() % p.n_kvblocks;
+      kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+    }
     float m = -INFINITY;  // running maximum, log2 domain (identical in the four parts)
     float l = 0.f;        // this part's running denominator
     bool ok = true;
-    // Keys of the current block from this tile on (blocks in ring order, as key_tile).
-    int kb_blk = group_of_cta() % p.n_kvblocks;
-    int kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
     for (int j = 0; j < ntiles; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, &g_attn_error, 30, kWaitLimitNs))) { ok = false; break; }
       if (threadIdx.x == 0) USP_TRACE_EV(5, j);
@@ -386,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_arrive(&bars->s_empty);
 
       float* s = reinterpret_cast<float*>(sr);
-      const int valid = kb_left - part * kCols;  // valid columns of this part (kb_left >= kBN: all)
+      int valid;  // valid columns of this part (>= kCols: all)
+      if constexpr (RING) valid = kb_left - part * kCols;
+      else valid = T - j * kBN - part * kCols;
       if (valid < kCols) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
@@ -477,10 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(&bars->p_full);
       if (threadIdx.x == 0) USP_TRACE_EV(9, j);
-      kb_left -= kBN;
-      if (kb_left <= 0) {
-        kb_blk = kb_blk == 0 ? p.n_kvblocks - 1 : kb_blk - 1;
-        kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+      if constexpr (RING) {
+        kb_left -= kBN;
+        if (kb_left <= 0) {
+          kb_blk = kb_blk == 0 ? p.n_kvblocks - 1 : kb_blk - 1;
+          kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+        }
       }
     }
     // Combine the four parts' denominators.
@@ -494,9 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort_flag, &g_attn_error, 33, kWaitLimitNs))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int g = group_of_cta();
-      const int t = first_row(g) + row;
-      const bool row_ok = t < p.q_start[g + 1] && t < T;
+      int t = qtile * kBM + row;
+      bool row_ok = t < T;
+      if constexpr (RING) {
+        const int g = group_of_cta();
+        t = first_row(g) + row;
+        row_ok = t < p.q_start[g + 1] && t < T;
+      }
       if (p.lse != nullptr && part == 0 && row_ok)  // sum_j exp(scale s_j) = 2^m * l
         p.lse[(static_cast<int64_t>(hm) * p.batch + b) * T + t] = (m + log2f(l)) * 0.69314718055994531f;
       const AttnOut& out = p.out;
@@ -593,15 +621,19 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   static_assert(C::SMEM_BYTES <= 232448, "shared memory above the 227 KB per-CTA limit");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(attention smem)");
+    for (auto* fn : {attn_tc_kernel<D, BF16, false>, attn_tc_kernel<D, BF16, true>}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(attention smem)");
+    }
     configured = true;
   }
   TcParams p;
   memset(&p, 0, sizeof(p));
   int rc;
   const int kv_tokens = L.kv_tokens > 0 ? L.kv_tokens : L.tokens;
+  const bool ring = L.blocks.n_qgroups > 0 || L.blocks.n_kvblocks > 0;
+  if (!ring && kv_tokens != L.tokens)
+    return set_error(USP_ERR_INVALID_ARG, "internal: the plain attention kernel takes as many keys as queries");
   if ((rc = make_map(&p.tm_q, L.in.q, L.in.qv, L, L.tokens, C::ATOM, kBM)) != USP_OK) return rc;
   if ((rc = make_map(&p.tm_k, L.in.k, L.in.kvv, L, kv_tokens, C::ATOM, kBN)) != USP_OK) return rc;
   if ((rc = make_map(&p.tm_v, L.in.v, L.in.kvv, L, kv_tokens, C::ATOM, kBN / 2)) != USP_OK) return rc;
@@ -619,7 +651,10 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   p.scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
   for (int i = 0; i < L.n_heads; ++i) p.heads[i] = L.heads[i];
   dim3 grid(p.q_tile_prefix[p.n_qgroups], L.batch * L.n_heads);
-  attn_tc_kernel<D, BF16><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  if (ring)
+    attn_tc_kernel<D, BF16, true><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  else
+    attn_tc_kernel<D, BF16, false><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   count_launch();
   return cuda_check(cudaGetLastError(), "attention (tcgen05) launch");
 }
