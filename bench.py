@@ -390,36 +390,69 @@ def run_ours(args, w, rank, world, local_rank):
             "gpu_launches": int(launches),
             "clocks": clk,
         }
-    # end-to-end through the public API with host buffers
+    # end-to-end through the public API with host buffers: every step copies
+    # its q/k/v in from pinned host memory and its output back. The copies run
+    # as a double-buffered pipeline on their own streams (inputs of step i+1
+    # come in and the output of step i-1 goes out while step i computes), the
+    # way a caller streaming batches from host memory would run them; the
+    # timed region spans the first input copy to the last output copy.
     if not args.no_e2e:
         host_in = [torch.from_numpy(x.view(np.int16) if w.dtype == "bf16" else x).pin_memory() for x in storage]
         host_out = torch.empty(full_out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
-        k_e2e = max(1, min(args.steps, 5))
+        k_e2e = max(2, args.steps)
+        fins = [full, [torch.empty_like(x) for x in full]]
+        fouts = [full_out, torch.empty_like(full_out)]
+        s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            for h, d in zip(host_in, full):
-                d.view(h.dtype).copy_(h, non_blocking=True)
-            if graphs:
-                graphs[0].replay()
-            else:
-                step()
-            host_out.copy_(full_out.view(host_out.dtype), non_blocking=True)
+        def step_on(fi, fo):
+            for x, sh in zip(fi, shards):
+                usp.scatter_sequence(plan, x, out=sh)
+            usp.ulysses_attention(plan, *shards, out=out, num_chunks=n_chunks, workspace=ws)
+            usp.gather_sequence(plan, out, out=fo)
 
-        e2e_step()
+        def e2e_run(nsteps):
+            ev = lambda: torch.cuda.Event()  # noqa: E731
+            h2d_done = [ev() for _ in range(nsteps)]
+            comp_done = [ev() for _ in range(nsteps)]
+            d2h_done = [ev() for _ in range(nsteps)]
+            s_h2d.wait_stream(stream)
+            s_d2h.wait_stream(stream)
+            for i in range(nsteps):
+                b = i % 2
+                with torch.cuda.stream(s_h2d):
+                    if i >= 2:
+                        s_h2d.wait_event(comp_done[i - 2])  # step i-2 has read input buffer b
+                    for h, d in zip(host_in, fins[b]):
+                        d.view(h.dtype).copy_(h, non_blocking=True)
+                    h2d_done[i].record(s_h2d)
+                stream.wait_event(h2d_done[i])
+                if i >= 2:
+                    stream.wait_event(d2h_done[i - 2])  # output buffer b has been copied out
+                step_on(fins[b], fouts[b])
+                comp_done[i].record(stream)
+                with torch.cuda.stream(s_d2h):
+                    s_d2h.wait_event(comp_done[i])
+                    host_out.copy_(fouts[b].view(host_out.dtype), non_blocking=True)
+                    d2h_done[i].record(s_d2h)
+            stream.wait_stream(s_d2h)
+            stream.wait_stream(s_h2d)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
+        e2e_run(k_e2e)
         e1.record(stream)
         torch.cuda.synchronize()
         (te_max,) = reduce_max([e0.elapsed_time(e1)], world, dev)
         if rank == 0:
             line["e2e"] = {"value": job_throughput(flop, k_e2e, te_max, world), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": 3 * w.tensor_bytes, "d2h_bytes_per_step": w.tensor_bytes,
-                           "steps": k_e2e}
-        del host_in, host_out
+                           "steps": k_e2e, "ms_per_step": te_max / k_e2e,
+                           "pipeline": "double-buffered: H2D of step i+1 and D2H of step i-1 overlap step i "
+                                       "on separate streams; timed from the first H2D to the last D2H"}
+        del host_in, host_out, fins, fouts
     del graphs
     plan.close()
     del full, shards, out, full_out, ws
