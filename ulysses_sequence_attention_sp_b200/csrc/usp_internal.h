@@ -191,6 +191,12 @@ inline bool fill_blocks(const AttnLaunch& L, int kv_tokens, int rows_per_tile, i
   return true;
 }
 
+// 4-D TMA map (d, head, token, batch) of one 16-bit attention operand view
+// with `rows` tokens; boxes of `atom` elements x 1 head x box_rows tokens,
+// swizzled by the atom width (64: 128 B, 32: 64 B, 16: 32 B).
+int make_map(CUtensorMap* map, const void* base, const AttnView& view, const AttnLaunch& L, int64_t rows, int atom,
+             int box_rows);
+
 bool attention_tc_supported(int dtype, int head_dim);
 int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream);
 int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream);
