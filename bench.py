@@ -496,6 +496,9 @@ def reshard_measurement(usp, torch, dev, pk, pk_kind):
         "all_gather_rows": (lambda: usp.all_gather_rows(plan, rows_local, out=rows_full), (1 + w.world) * S),
         "reduce_scatter_rows": (lambda: usp.reduce_scatter_rows(plan, rows_full, out=rows_out), (w.world + 1) * S),
     }
+    tma_plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix)
+    tma_plan.set_pack_mode("tma")
+    ops["seq_to_head_qkv_tma"] = (lambda: usp.ulysses_seq_to_head(tma_plan, seq, out=heads), 6 * S)
     res = {}
     for name, (fn, nbytes) in ops.items():
         for _ in range(2):
@@ -512,6 +515,7 @@ def reshard_measurement(usp, torch, dev, pk, pk_kind):
     usp.ulysses_head_to_seq(plan, heads, out=seq)
     torch.cuda.synchronize()
     plan.close()
+    tma_plan.close()
     s2h = res["seq_to_head_qkv"]
     return {"workload": w.name, "ops": res, "peak_gbs": pk["hbm_gbs"], "peak_source": f"hbm_gbs ({pk_kind})",
             "roofline": {"bound": "hbm", "achieved": s2h["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -150,6 +150,21 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
                            int32_t head_dim, int32_t ulysses_size, int32_t ring_size, int32_t dtype,
                            int32_t prefix_tokens);
 
+/*
+ * usp_plan_set_pack_mode -- how this plan's sequence -> head moves
+ * (usp_ulysses_seq_to_head(_kv) and the pack inside usp_ulysses_attention)
+ * run. USP_PACK_VECTOR (the default): 16-byte vector loads and stores, one
+ * warp per sequence row. USP_PACK_TMA: TMA tile copies, global -> shared ->
+ * global, one head unit of up to 64 rows per tile, no multicast; used where a
+ * head unit (head_dim * element size) is a multiple of 16 bytes of at most
+ * 256 elements, the vector kernel otherwise. Both give identical bytes
+ * ("h3_blackwell_runtime/distributed.py", seq_to_heads). Errors:
+ * USP_ERR_INVALID_ARG for an unknown mode.
+ */
+#define USP_PACK_VECTOR 0
+#define USP_PACK_TMA 1
+int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode);
+
 /* Copies the plan's Ulysses group size and ring size out (world and 1 for a plain plan); either may be NULL. */
 int usp_plan_query_hybrid(const usp_plan* plan, int32_t* ulysses_size, int32_t* ring_size);
 

@@ -73,9 +73,14 @@ def _run_layout_checks(usp, plan, itemsize, seed, ntensors=1):
     assert usp.device_status() == 0
 
 
+MODES = ["vector", "tma"]  # how sequence -> head moves run (16-byte vectors or TMA tile copies)
+
+
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("w", ALL, ids=[w.name for w in ALL])
-def test_layout_full_size(usp, w):
+def test_layout_full_size(usp, w, mode):
     with usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix) as plan:
+        plan.set_pack_mode(mode)
         _run_layout_checks(usp, plan, w.elem_bytes, seed=2000 + w.seed % 1000)
 
 
@@ -94,10 +99,12 @@ SMALL = [  # batch, seq_len, heads, head_dim, world, dtype, prefix, ntensors
 ]
 
 
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("case", SMALL)
-def test_layout_small_ragged(usp, case):
+def test_layout_small_ragged(usp, case, mode):
     batch, seq_len, heads, dim, world, dtype, prefix, nt = case
     with usp.Plan(batch, seq_len, heads, dim, world, dtype, prefix) as plan:
+        plan.set_pack_mode(mode)
         itemsize = 4 if dtype == "fp32" else 2
         if (heads * dim * itemsize) % 16:
             # scatter/gather need 16-byte rows; the exchanges do not

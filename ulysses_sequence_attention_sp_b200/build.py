@@ -24,7 +24,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG_DIR, "libusp.so")
 
-SOURCES = ["plan.cpp", "tensor_map.cpp", "permute.cu", "rows.cu", "attn_tc.cu", "attn_simt.cu", "noalloc.cu"]
+SOURCES = ["plan.cpp", "tensor_map.cpp", "permute.cu", "pack_tma.cu", "rows.cu", "attn_tc.cu", "attn_simt.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           f"-I{INCLUDE}", f"-I{CSRC}"]

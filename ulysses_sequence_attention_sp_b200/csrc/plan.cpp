@@ -127,6 +127,14 @@ void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) 
     }
 }
 
+// A sequence -> head move: TMA tile copies when the plan asks for them and the
+// head unit allows it (a multiple of 16 bytes), else 16-byte vector copies.
+int launch_pack(const usp_plan* plan, const usp::PermuteArgs& a, int vec, int64_t unit, cudaStream_t stream) {
+  if (a.dir == 0 && plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit))
+    return usp::launch_pack_tma(a, plan->elem, unit, stream);
+  return usp::launch_permute(a, vec, stream);
+}
+
 // kv selects the k/v head geometry (Hkv heads split by kv_head_start) instead
 // of the query geometry.
 int seq_head_exchange(const usp_plan* plan, int dir, int32_t ntensors, const void* const* seq, void* const* heads,
@@ -152,7 +160,7 @@ int seq_head_exchange(const usp_plan* plan, int dir, int32_t ntensors, const voi
       a.seq_ptr[t][r] = const_cast<void*>(seq[t * plan->world + r]);
       a.head_ptr[t][r] = heads[t * plan->world + r];
     }
-  return usp::launch_permute(a, vec, stream);
+  return launch_pack(plan, a, vec, unit, stream);
 }
 
 }  // namespace
@@ -776,10 +784,10 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   const cudaStream_t ps = overlap ? plan->aux : s;
   for (int c = 0; c < nchunks; ++c) {
     select_chunk_heads(aq, plan, lo[c], hi[c]);
-    if (int rc = usp::launch_permute(aq, vec, ps)) return rc;
+    if (int rc = launch_pack(plan, aq, vec, unit, ps)) return rc;
     if (gqa) {
       select_chunk_kv_heads(akv, plan, lo[c], hi[c]);
-      if (int rc = usp::launch_permute(akv, vec, ps)) return rc;
+      if (int rc = launch_pack(plan, akv, vec, unit, ps)) return rc;
     }
     if (overlap) {
       if (int rc = usp::cuda_check(cudaEventRecord(plan->ev_chunk[c], plan->aux), "cudaEventRecord")) return rc;
@@ -793,6 +801,14 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   }
   if (plan->t_stop)
     if (int rc = record_timing_event(plan->t_stop, s)) return rc;
+  return USP_OK;
+}
+
+int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode) {
+  if (int rc = check_plan(plan)) return rc;
+  if (mode != USP_PACK_VECTOR && mode != USP_PACK_TMA)
+    return usp::set_error(USP_ERR_INVALID_ARG, "pack mode must be USP_PACK_VECTOR or USP_PACK_TMA (got %d)", mode);
+  plan->pack_mode = mode;
   return USP_OK;
 }
 
@@ -812,6 +828,9 @@ int usp_device_status(uint32_t* code, int32_t reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return usp::cuda_check(e, "cudaDeviceSynchronize");
   if (int rc = usp::read_attention_error(code, reset != 0)) return rc;
+  uint32_t pack_code = 0;
+  if (int rc = usp::read_pack_error(&pack_code, reset != 0)) return rc;
+  if (*code == 0) *code = pack_code;
   if (*code != 0) {
     usp::set_error(USP_ERR_TIMEOUT, "a device-side wait ran out (site %u)", *code);
     return USP_ERR_TIMEOUT;

@@ -32,6 +32,7 @@ struct usp_plan {
   // consecutive ranks. The plain block is head_ranks == world, ring == 1.
   int32_t head_ranks = 0;
   int32_t ring = 1;
+  int32_t pack_mode = 0;  // USP_PACK_VECTOR or USP_PACK_TMA: how seq->head packs move data
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
@@ -78,6 +79,13 @@ struct PermuteArgs {
 
 // vec_bytes in {16, 8, 4, 2}; dv counts vectors of that size.
 int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream);
+
+// The same sequence -> head permutation (dir 0) moved by TMA tile copies
+// (pack_tma.cu); unit_bytes = bytes of one head unit. Needs 2- or 4-byte
+// elements and unit_bytes a multiple of 16 of at most 256 elements.
+bool pack_tma_supported(int elem, int64_t unit_bytes);
+int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStream_t stream);
+int read_pack_error(uint32_t* code, bool reset);
 
 int sm_count();
 

@@ -72,6 +72,7 @@ _SIGNATURES = {
     "usp_ulysses_attention_lse": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_void_p,
                                                  ctypes.c_float, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                                  ctypes.c_void_p]),
+    "usp_plan_set_pack_mode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
     "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
     "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
@@ -252,6 +253,14 @@ class Plan:
         if fill is not None:
             t.fill_(fill)
         return t
+
+    def set_pack_mode(self, mode: str) -> None:
+        """'vector' (default) or 'tma': how sequence -> head moves run (same bytes)."""
+        codes = {"vector": 0, "tma": 1}
+        if mode not in codes:
+            raise UspError(USP_ERR_INVALID_ARG, f"pack mode must be one of {sorted(codes)}")
+        _check(_lib.usp_plan_set_pack_mode(self.handle, codes[mode]))
+        self.pack_mode = mode
 
     def workspace_bytes(self, num_chunks: int = 1) -> int:
         n = ctypes.c_size_t()
