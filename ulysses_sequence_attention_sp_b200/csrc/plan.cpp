@@ -14,11 +14,22 @@
 #include <atomic>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "usp_internal.h"
 
 namespace {
 
 thread_local std::string g_last_error;
+
+// NVTX range over one host call or step (the CPU side of a profiler timeline;
+// free when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -399,6 +410,7 @@ static int scatter_gather(const usp_plan* plan, int dir, const void* full, void*
 
 int usp_scatter_sequence(const usp_plan* plan, const void* x_full, void* const* x_shards, int64_t outer,
                          int64_t row_bytes, void* stream) {
+  NvtxRange range("usp_scatter_sequence");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(x_shards), plan->world, "x_shards")) return rc;
@@ -408,6 +420,7 @@ int usp_scatter_sequence(const usp_plan* plan, const void* x_full, void* const* 
 
 int usp_gather_sequence(const usp_plan* plan, const void* const* x_shards, void* x_full, int64_t outer,
                         int64_t row_bytes, void* stream) {
+  NvtxRange range("usp_gather_sequence");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
   if (int rc = check_ptrs(x_shards, plan->world, "x_shards")) return rc;
@@ -448,6 +461,7 @@ static int head_slice_gather(const usp_plan* plan, int dir, const void* full, vo
 
 int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards, int64_t rows,
                       void* stream) {
+  NvtxRange range("usp_sp_head_slice");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_sp_head_slice")) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
@@ -458,6 +472,7 @@ int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_h
 
 int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, void* x_full, int64_t rows,
                        void* stream) {
+  NvtxRange range("usp_sp_head_gather");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_sp_head_gather")) return rc;
   if (int rc = check_ptr(x_full, "x_full")) return rc;
@@ -470,6 +485,7 @@ int usp_sp_head_gather(const usp_plan* plan, const void* const* x_head_shards, v
 // Row collectives: the plan's token split, `outer` batches, rows of row_bytes.
 static int rows_collective(const usp_plan* plan, bool reduce, const void* const* src, void* const* dst,
                            int64_t outer, int64_t row_bytes, void* stream) {
+  NvtxRange range(reduce ? "usp_reduce_scatter_rows" : "usp_all_gather_rows");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_ptrs(src, plan->world, reduce ? "partial_full_rows" : "local_rows")) return rc;
   if (int rc = check_ptrs(const_cast<const void* const*>(dst), plan->world, reduce ? "local_rows" : "full_rows"))
@@ -511,6 +527,7 @@ int usp_reduce_scatter_rows(const usp_plan* plan, const void* const* partial_ful
 
 int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
+  NvtxRange range("usp_ulysses_seq_to_head");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_ulysses_seq_to_head")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
@@ -522,6 +539,7 @@ int usp_ulysses_seq_to_head(const usp_plan* plan, int32_t ntensors, const void* 
 
 int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                                void* stream) {
+  NvtxRange range("usp_ulysses_seq_to_head_kv");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_ulysses_seq_to_head_kv")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
@@ -533,6 +551,7 @@ int usp_ulysses_seq_to_head_kv(const usp_plan* plan, int32_t ntensors, const voi
 
 int usp_ulysses_head_to_seq(const usp_plan* plan, int32_t ntensors, const void* const* in, void* const* out,
                             void* stream) {
+  NvtxRange range("usp_ulysses_head_to_seq");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_ulysses_head_to_seq")) return rc;
   if (ntensors < 1 || ntensors > 3) return usp::set_error(USP_ERR_INVALID_ARG, "ntensors must be 1..3");
@@ -564,6 +583,7 @@ static float resolve_scale(const usp_plan* plan, float scale) {
 
 int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const void* const* k_heads,
                        const void* const* v_heads, void* const* o_heads, float scale, void* stream) {
+  NvtxRange range("usp_head_attention");
   if (int rc = check_plan(plan)) return rc;
   if (int rc = check_flat(plan, "usp_head_attention")) return rc;
   if (int rc = check_ptrs(q_heads, plan->world, "q_heads")) return rc;
@@ -672,6 +692,7 @@ int usp_ulysses_attention_lse(const usp_plan* plan, const void* const* q, const 
 static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, const void* const* k,
                                   const void* const* v, void* const* out, float* lse, float scale, int32_t num_chunks,
                                   void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("usp_ulysses_attention");
   if (int rc = check_plan(plan)) return rc;
   if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive (got %d)", num_chunks);
   if (int rc = check_ptrs(q, plan->world, "q")) return rc;
@@ -783,6 +804,9 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   }
   const cudaStream_t ps = overlap ? plan->aux : s;
   for (int c = 0; c < nchunks; ++c) {
+    char range_name[64];
+    snprintf(range_name, sizeof(range_name), "usp chunk %d/%d: pack + attention", c + 1, nchunks);
+    NvtxRange chunk_range(range_name);
     select_chunk_heads(aq, plan, lo[c], hi[c]);
     if (int rc = launch_pack(plan, aq, vec, unit, ps)) return rc;
     if (gqa) {
