@@ -55,7 +55,9 @@ enum usp_status {
   USP_ERR_CUDA = 5,        /* a CUDA runtime call failed (message has the name)    */
   USP_ERR_TIMEOUT = 6,     /* a device-side wait ran out (see usp_device_status)  */
   USP_ERR_UNSUPPORTED = 7, /* valid but not built (e.g. head_dim > 256)           */
-  USP_ERR_NO_DEVICE = 8    /* no CUDA device is visible                           */
+  USP_ERR_NO_DEVICE = 8,   /* no CUDA device is visible                           */
+  USP_ERR_BOUNDS = 9       /* a bounds-checking build (-DUSP_BOUNDS_CHECK) skipped an
+                              out-of-range offset (see usp_device_status)          */
 };
 
 enum usp_dtype { USP_BF16 = 0, USP_FP32 = 1, USP_FP16 = 2 };
@@ -361,9 +363,11 @@ uint64_t usp_kernel_launches(void);
 
 /*
  * usp_device_status -- synchronises the current device, then reads the
- * library's device-side error word of its kernels (0 = no error; nonzero =
- * a bounded device-side wait ran out, and identifies the wait). reset != 0
- * clears it. Diagnostic only.
+ * library's device-side error words (0 = no error). A bounded device-side
+ * wait that ran out returns USP_ERR_TIMEOUT with *code = the wait's site; in
+ * a bounds-checking build (-DUSP_BOUNDS_CHECK), an out-of-range offset that a
+ * kernel skipped returns USP_ERR_BOUNDS with *code = the access site. reset
+ * != 0 clears the words. Diagnostic only.
  */
 int usp_device_status(uint32_t* code, int32_t reset);
 

@@ -23,6 +23,10 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG_DIR, "libusp.so")
+# The bounds-checking build (-DUSP_BOUNDS_CHECK): every global offset of the copy
+# kernels and the attention epilogues is range-checked; a debugging aid, loaded
+# through $USP_LIBRARY.
+CHECKED_LIB_PATH = os.path.join(PKG_DIR, "libusp_checked.so")
 
 SOURCES = ["plan.cpp", "tensor_map.cpp", "permute.cu", "pack_tma.cu", "rows.cu", "attn_tc.cu", "attn_simt.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -84,6 +88,14 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("linking libusp.so failed")
     os.replace(tmp, lib_path)
     return lib_path
+
+
+def build_checked(force: bool = False, verbose: bool = False) -> str:
+    """Builds the bounds-checking variant into CHECKED_LIB_PATH; returns its path."""
+    if (not force and os.path.exists(CHECKED_LIB_PATH)
+            and all(os.path.getmtime(f) <= os.path.getmtime(CHECKED_LIB_PATH) for f in _deps())):
+        return CHECKED_LIB_PATH
+    return build(force=True, verbose=verbose, extra=["-DUSP_BOUNDS_CHECK"], out=CHECKED_LIB_PATH)
 
 
 def main() -> None:

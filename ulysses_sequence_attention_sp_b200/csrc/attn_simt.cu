@@ -10,9 +10,13 @@
 #include <cmath>
 
 #include "device_common.cuh"
+#include "bounds_check.cuh"
 #include "usp_internal.h"
 
 namespace usp {
+
+__device__ uint32_t g_simt_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
+
 namespace {
 
 constexpr int kTPR = 4;                  // threads per query row
@@ -103,8 +107,11 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
     m = m_new;
   }
   if (!row_ok) return;
-  if (L.lse != nullptr && sub == 0)  // sum_j exp(scale s_j) = 2^m * l
-    L.lse[(static_cast<int64_t>(hm) * L.batch + b) * T + row] = (m + log2f(l)) * 0.69314718055994531f;
+  if (L.lse != nullptr && sub == 0) {  // sum_j exp(scale s_j) = 2^m * l
+    const int64_t li = (static_cast<int64_t>(hm) * L.batch + b) * T + row;
+    if (in_bounds(li, 1, static_cast<int64_t>(L.in.qv.head_extent) * L.batch * T, 42, &g_simt_bounds))
+      L.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
+  }
 
   const AttnOut& out = L.out;
   int seg_lo, seg_hi;
@@ -124,11 +131,13 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
   const float inv_l = 1.f / l;
   for (int s = seg_lo; s < seg_hi; ++s) {
     const int64_t rows_s = out.prefix + out.seg_len[s];
-    float* dst = static_cast<float*>(out.seg_ptr[s]) + ((b * rows_s + row_in_seg) * out.out_heads + hm) * D;
+    const int64_t base = ((b * rows_s + row_in_seg) * out.out_heads + hm) * D;
+    float* dst = static_cast<float*>(out.seg_ptr[s]) + base;
+    const int64_t ext = static_cast<int64_t>(L.batch) * rows_s * out.out_heads * D;  // bounds-checking builds
 #pragma unroll
     for (int i = 0; i < DPT; ++i) {
       const int d = sub * DPT + i;
-      if (d < D) dst[d] = acc[i] * inv_l;
+      if (d < D && in_bounds(base + d, 1, ext, 41, &g_simt_bounds)) dst[d] = acc[i] * inv_l;
     }
   }
 }
@@ -164,6 +173,17 @@ int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream) {
   if (D <= 128) return launch_dpt<32>(L, stream);
   if (D <= 256) return launch_dpt<64>(L, stream);
   return set_error(USP_ERR_UNSUPPORTED, "head_dim %d > 256 is not built", D);
+}
+
+int read_simt_bounds(uint32_t* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_simt_bounds, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_check(e, "read fp32 attention bounds word");
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_simt_bounds, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_check(e, "reset fp32 attention bounds word");
+  }
+  return USP_OK;
 }
 
 }  // namespace usp

@@ -46,11 +46,13 @@
 #include <cuda_fp16.h>
 
 #include "device_common.cuh"
+#include "bounds_check.cuh"
 #include "usp_internal.h"
 
 namespace usp {
 
-__device__ uint32_t g_attn_error;  // first wait that ran out (site code), 0 if none
+__device__ uint32_t g_attn_error;   // first wait that ran out (site code), 0 if none
+__device__ uint32_t g_attn_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
 
 // Pipeline trace (built only with -DUSP_TRACE): clock64() at pipeline events
 // of one CTA, [event][key tile]; read with usp_debug_read_trace.
@@ -122,7 +124,8 @@ static_assert(sizeof(Bars) + 8 <= 5120, "barrier block outgrew its shared-memory
 struct TcParams {
   CUtensorMap tm_q, tm_k, tm_v;   // boxes: Q 128 rows, K 256 rows, V 128 rows
   AttnOut out;
-  float* lse;
+  float* lse;                     // optional [head][batch][tokens], natural log
+  int64_t lse_ext;                // its elements (bounds-checking builds)
   int32_t tokens, batch, n_heads, kv_tokens;
   int32_t kv_group, q_head_base, kv_head_base, pad1;  // k/v head of query head h: (q_head_base + h) / kv_group - kv_head_base
   float scale_log2;
@@ -524,8 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         t = first_row(g) + row;
         row_ok = t < p.q_start[g + 1] && t < T;
       }
-      if (p.lse != nullptr && part == 0 && row_ok)  // sum_j exp(scale s_j) = 2^m * l
-        p.lse[(static_cast<int64_t>(hm) * p.batch + b) * T + t] = (m + log2f(l)) * 0.69314718055994531f;
+      if (p.lse != nullptr && part == 0 && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
+        const int64_t li = (static_cast<int64_t>(hm) * p.batch + b) * T + t;
+        if (in_bounds(li, 1, p.lse_ext, 22, &g_attn_bounds)) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
+      }
       const AttnOut& out = p.out;
       // Destination(s) of this row.
       int seg_lo = 0, seg_hi = 0;
@@ -560,6 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int sg = seg_lo; sg < seg_hi; ++sg) {
           const int64_t rows_s = out.prefix + out.seg_len[sg];
           const int64_t elem = ((static_cast<int64_t>(b) * rows_s + row_in_seg) * out.out_heads + hm) * D + c * 16;
+          if (!in_bounds(elem, 16, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 21, &g_attn_bounds))
+            continue;
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem);
           dst[0] = w0;
           dst[1] = w1;
@@ -603,6 +610,7 @@ int launch_d(const AttnLaunch& L, cudaStream_t stream) {
     return set_error(USP_ERR_INVALID_ARG, "internal: bad query-group or key-block table");
   p.kv_tokens = kv_tokens;
   p.lse = L.lse;
+  p.lse_ext = static_cast<int64_t>(L.in.qv.head_extent) * L.batch * L.tokens;
   p.kv_group = L.in.kv_group;
   p.q_head_base = L.in.q_head_base;
   p.kv_head_base = L.in.kv_head_base;
@@ -659,6 +667,17 @@ bool attention_tc_supported(int dtype, int head_dim) {
 int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream) {
   if (L.n_heads == 0 || L.batch == 0 || L.tokens == 0) return USP_OK;
   return L.dtype == USP_BF16 ? launch_dtype<true>(L, stream) : launch_dtype<false>(L, stream);
+}
+
+int read_attention_bounds(uint32_t* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_attn_bounds, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_check(e, "read attention bounds word");
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_attn_bounds, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_check(e, "reset attention bounds word");
+  }
+  return USP_OK;
 }
 
 int read_attention_error(uint32_t* code, bool reset) {

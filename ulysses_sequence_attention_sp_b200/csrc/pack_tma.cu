@@ -16,11 +16,13 @@
 // (the overlapped rows are written twice with the same bytes).
 // No multicast: every load reads this device's own memory into its own CTA.
 #include "device_common.cuh"
+#include "bounds_check.cuh"
 #include "usp_internal.h"
 
 namespace usp {
 
-__device__ uint32_t g_pack_error;  // first wait that ran out (site code), 0 if none
+__device__ uint32_t g_pack_error;   // first wait that ran out (site code), 0 if none
+__device__ uint32_t g_pack_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
 
 namespace {
 
@@ -48,6 +50,9 @@ struct PackTmaParams {
   int32_t cnt[USP_MAX_WORLD];            // its row count
   int32_t d0[USP_MAX_WORLD];             // token offset of its first row on the head side
   int32_t chunk_prefix[USP_MAX_WORLD + 1];
+  int32_t heads;                         // head units per sequence row (bounds-checking builds)
+  int32_t buf_heads[USP_MAX_WORLD];      // head units of each head-side buffer
+  int32_t full_tokens;                   // token rows of each head-side buffer
   uint16_t sel_head[USP_MAX_HEADS];      // head unit in the sequence row
   uint16_t sel_local[USP_MAX_HEADS];     // its index inside the owning head-side buffer
   uint8_t sel_rank[USP_MAX_HEADS];       // the owning head-side buffer
@@ -109,6 +114,10 @@ __global__ void __launch_bounds__(32, 1) pack_tma_kernel(const __grid_constant__
   auto load = [&](int64_t k) {
     const Unit u = unit_of(p, first + k * step);
     const int st = static_cast<int>(k % kStages);
+    // bounds-checking builds: the tile stays inside the source rank's rows and heads
+    // (the copy still runs, so the mbarrier completes; the site is recorded)
+    in_bounds(u.row, p.rows, p.r0[u.s] + p.cnt[u.s], 61, &g_pack_bounds);
+    in_bounds(p.sel_head[u.i], p.hb, p.heads, 62, &g_pack_bounds);
     mbar_arrive_expect_tx(&full[st], p.box_bytes);
     tma_load_4d(&p.src[u.t][u.s], &full[st], smem + static_cast<size_t>(st) * p.stage_bytes, 0, p.sel_head[u.i],
                 u.row, u.b);
@@ -123,9 +132,15 @@ __global__ void __launch_bounds__(32, 1) pack_tma_kernel(const __grid_constant__
       break;
     fence_proxy_async_smem();  // the landed tile, seen by this thread, before the store reads it
     const Unit u = unit_of(p, first + k * step);
-    tma_store_4d(&p.dst[u.t][p.sel_rank[u.i]], smem + static_cast<size_t>(st) * p.stage_bytes, 0,
-                 p.sel_local[u.i], u.tok, u.b);
-    bulk_commit_group();
+    if (!in_bounds(u.tok, p.rows, p.d0[u.s] + p.cnt[u.s], 63, &g_pack_bounds) ||
+        !in_bounds(p.sel_local[u.i], p.hb, p.buf_heads[p.sel_rank[u.i]], 64, &g_pack_bounds) ||
+        !in_bounds(u.tok, p.rows, p.full_tokens, 65, &g_pack_bounds)) {
+      bulk_commit_group();  // an empty group keeps the stage accounting of wait_group.read
+    } else {
+      tma_store_4d(&p.dst[u.t][p.sel_rank[u.i]], smem + static_cast<size_t>(st) * p.stage_bytes, 0,
+                   p.sel_local[u.i], u.tok, u.b);
+      bulk_commit_group();
+    }
     if (issued < mine) {
       bulk_wait_group_read_1();  // the store of unit k-1 has read its stage, which the next load reuses
       load(issued);
@@ -233,6 +248,9 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
     p.sel_local[i] = static_cast<uint16_t>(a.sel_head[i] - a.head_start[a.sel_rank[i]]);
   }
   p.total_units = static_cast<int64_t>(a.ntensors) * a.outer * p.chunk_prefix[a.n_seq] * p.ngroups;
+  p.heads = a.heads;
+  p.full_tokens = static_cast<int32_t>(a.full_tokens);
+  for (int r = 0; r < a.n_head; ++r) p.buf_heads[r] = a.head_start[r + 1] - a.head_start[r];
   int rc;
   for (int t = 0; t < a.ntensors; ++t) {
     for (int s = 0; s < a.n_seq; ++s) {
@@ -266,6 +284,17 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
   pack_tma_kernel<<<grid, 32, smem, stream>>>(p);
   count_launch();
   return cuda_check(cudaGetLastError(), "TMA pack launch");
+}
+
+int read_pack_bounds(uint32_t* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_pack_bounds, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_check(e, "read pack bounds word");
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_pack_bounds, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_check(e, "reset pack bounds word");
+  }
+  return USP_OK;
 }
 
 int read_pack_error(uint32_t* code, bool reset) {

@@ -14,9 +14,12 @@
 #include <cstdio>
 
 #include "device_common.cuh"
+#include "bounds_check.cuh"
 #include "usp_internal.h"
 
 namespace usp {
+__device__ uint32_t g_permute_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -90,18 +93,20 @@ __global__ void __launch_bounds__(kThreads, 4) permute_kernel(const __grid_const
           const V* src = static_cast<const V*>(a.seq_ptr[ti][s]);
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u)
-            if (ok[u]) val[u] = __ldcs(src + soff[u]);
+            if (ok[u] && in_bounds(soff[u], 1, a.seq_ext[s], 1, &g_permute_bounds)) val[u] = __ldcs(src + soff[u]);
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u)
-            if (ok[u]) __stcs(static_cast<V*>(a.head_ptr[ti][hr[u]]) + hoff[u], val[u]);
+            if (ok[u] && in_bounds(hoff[u], 1, a.head_ext[hr[u]], 2, &g_permute_bounds))
+              __stcs(static_cast<V*>(a.head_ptr[ti][hr[u]]) + hoff[u], val[u]);
         } else {
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u)
-            if (ok[u]) val[u] = __ldcs(static_cast<const V*>(a.head_ptr[ti][hr[u]]) + hoff[u]);
+            if (ok[u] && in_bounds(hoff[u], 1, a.head_ext[hr[u]], 3, &g_permute_bounds))
+              val[u] = __ldcs(static_cast<const V*>(a.head_ptr[ti][hr[u]]) + hoff[u]);
           V* dst = static_cast<V*>(a.seq_ptr[ti][s]);
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u)
-            if (ok[u]) __stcs(dst + soff[u], val[u]);
+            if (ok[u] && in_bounds(soff[u], 1, a.seq_ext[s], 4, &g_permute_bounds)) __stcs(dst + soff[u], val[u]);
         }
       }
     }
@@ -122,6 +127,9 @@ int sm_count() {
 
 int launch_permute(const PermuteArgs& args, int vec_bytes, cudaStream_t stream) {
   PermuteArgs a = args;
+  for (int s = 0; s < a.n_seq; ++s) a.seq_ext[s] = (a.seq_rows[s + 1] - a.seq_rows[s]) * a.heads * a.dv;
+  for (int r = 0; r < a.n_head; ++r)
+    a.head_ext[r] = a.outer * a.full_tokens * (a.head_start[r + 1] - a.head_start[r]) * a.dv;
   const int64_t rows = a.seq_rows[a.n_seq];
   if (rows == 0 || a.nsel == 0) return USP_OK;
   // Several tensors per launch already make the launch long next to its tail:
@@ -156,6 +164,17 @@ int launch_permute(const PermuteArgs& args, int vec_bytes, cudaStream_t stream) 
   }
   count_launch();
   return cuda_check(cudaGetLastError(), "permute kernel launch");
+}
+
+int read_permute_bounds(uint32_t* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_permute_bounds, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_check(e, "read permute bounds word");
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_permute_bounds, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_check(e, "reset permute bounds word");
+  }
+  return USP_OK;
 }
 
 }  // namespace usp

@@ -859,6 +859,19 @@ int usp_device_status(uint32_t* code, int32_t reset) {
     usp::set_error(USP_ERR_TIMEOUT, "a device-side wait ran out (site %u)", *code);
     return USP_ERR_TIMEOUT;
   }
+  // Bounds-checking builds record the first out-of-range access per kernel file.
+  int (*const readers[])(uint32_t*, bool) = {usp::read_permute_bounds, usp::read_rows_bounds,
+                                             usp::read_pack_bounds, usp::read_attention_bounds,
+                                             usp::read_simt_bounds};
+  for (auto read : readers) {
+    uint32_t site = 0;
+    if (int rc = read(&site, reset != 0)) return rc;
+    if (*code == 0) *code = site;
+  }
+  if (*code != 0) {
+    usp::set_error(USP_ERR_BOUNDS, "an out-of-range offset was skipped (site %u)", *code);
+    return USP_ERR_BOUNDS;
+  }
   return USP_OK;
 }
 

@@ -19,9 +19,13 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "bounds_check.cuh"
 #include "usp_internal.h"
 
 namespace usp {
+
+__device__ uint32_t g_rows_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -54,17 +58,20 @@ __global__ void __launch_bounds__(kThreads) all_gather_rows_kernel(const __grid_
     const int64_t base = m.k * kTile + threadIdx.x;
     V val[kU];
     bool ok[kU];
+    const int64_t src_ext = a.outer * a.tok_len[m.r] * a.nv;  // bounds-checking builds only
+    const int64_t dst_ext = a.outer * a.total_rows * a.nv;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int64_t j = base + u * kThreads;
       ok[u] = j < seg_len;
-      if (ok[u]) val[u] = __ldcs(src + j);
+      if (ok[u] && in_bounds(m.b * seg_len + j, 1, src_ext, 11, &g_rows_bounds)) val[u] = __ldcs(src + j);
     }
     for (int d = 0; d < a.world; ++d) {
       V* dst = static_cast<V*>(a.dst[d]) + doff;
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        if (ok[u]) __stcs(dst + base + u * kThreads, val[u]);
+        if (ok[u] && in_bounds(doff + base + u * kThreads, 1, dst_ext, 12, &g_rows_bounds))
+          __stcs(dst + base + u * kThreads, val[u]);
     }
   }
 }
@@ -118,7 +125,8 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_rows_kernel(const __g
           const V* src = static_cast<const V*>(a.src[i0 + q]) + soff;
 #pragma unroll
           for (int u = 0; u < kU; ++u)
-            if (ok[u]) x[q][u].v = __ldcs(src + base + u * kThreads);
+            if (ok[u] && in_bounds(soff + base + u * kThreads, 1, a.outer * a.total_rows * a.nv, 13, &g_rows_bounds))
+              x[q][u].v = __ldcs(src + base + u * kThreads);
         }
       }
 #pragma unroll
@@ -134,7 +142,9 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_rows_kernel(const __g
     V* dst = static_cast<V*>(a.dst[m.r]) + m.b * seg_len;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      if (!ok[u]) continue;
+      if (!ok[u] ||
+          !in_bounds(m.b * seg_len + base + u * kThreads, 1, a.outer * a.tok_len[m.r] * a.nv, 14, &g_rows_bounds))
+        continue;
       Pack<V, E> o;
 #pragma unroll
       for (int e = 0; e < kE; ++e) o.e[e] = from_f32<E>(acc[u][e]);
@@ -222,6 +232,17 @@ int launch_reduce_scatter_rows(const RowsArgs& a, int vec_bytes, int dtype, cuda
     case USP_FP32: return reduce_e<float>(a, vec_bytes, s);
     default: return set_error(USP_ERR_DTYPE, "unknown dtype %d", dtype);
   }
+}
+
+int read_rows_bounds(uint32_t* code, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_rows_bounds, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_check(e, "read rows bounds word");
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_rows_bounds, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_check(e, "reset rows bounds word");
+  }
+  return USP_OK;
 }
 
 }  // namespace usp

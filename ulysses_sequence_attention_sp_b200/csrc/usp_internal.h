@@ -75,10 +75,20 @@ struct PermuteArgs {
   uint8_t sel_rank[USP_MAX_HEADS];        // head-side buffer owning each moved unit
   void* seq_ptr[3][USP_MAX_WORLD];
   void* head_ptr[3][USP_MAX_WORLD];
+  int64_t seq_ext[USP_MAX_WORLD];   // vectors in sequence-side buffer s (set by launch_permute)
+  int64_t head_ext[USP_MAX_WORLD];  // vectors in head-side buffer r (set by launch_permute)
 };
 
 // vec_bytes in {16, 8, 4, 2}; dv counts vectors of that size.
 int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream);
+
+// Bounds-checking builds: the first out-of-range site each copy kernel
+// recorded (0 if none), read and optionally reset, per translation unit.
+int read_permute_bounds(uint32_t* code, bool reset);
+int read_rows_bounds(uint32_t* code, bool reset);
+int read_attention_bounds(uint32_t* code, bool reset);
+int read_simt_bounds(uint32_t* code, bool reset);
+int read_pack_bounds(uint32_t* code, bool reset);
 
 // The same sequence -> head permutation (dir 0) moved by TMA tile copies
 // (pack_tma.cu); unit_bytes = bytes of one head unit. Needs 2- or 4-byte

@@ -32,6 +32,7 @@ USP_ERR_CUDA = 5
 USP_ERR_TIMEOUT = 6
 USP_ERR_UNSUPPORTED = 7
 USP_ERR_NO_DEVICE = 8
+USP_ERR_BOUNDS = 9
 
 USP_BF16, USP_FP32, USP_FP16 = 0, 1, 2
 MAX_WORLD = 32
@@ -499,10 +500,12 @@ def kernel_launches() -> int:
 
 
 def device_status(reset: bool = True) -> int:
-    """Synchronises the device and returns the library's device-side error word."""
+    """Synchronises the device and returns the library's device-side error word:
+    0, a wait's site (a wait ran out) or, in a bounds-checking build, the site
+    of a skipped out-of-range access."""
     code = ctypes.c_uint32()
     rc = _lib.usp_device_status(ctypes.byref(code), 1 if reset else 0)
-    if rc not in (USP_OK, USP_ERR_TIMEOUT):
+    if rc not in (USP_OK, USP_ERR_TIMEOUT, USP_ERR_BOUNDS):
         _check(rc)
     return code.value
 
