@@ -299,3 +299,41 @@ def test_block_replays_from_a_cuda_graph(usp, num_chunks):
     assert usp.device_status() == 0
     del graph
     plan.close()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_trivial_group_is_byte_identical_to_single_device(usp, dtype):
+    """API page, ulysses_attention: a one-rank group gives exactly the non-SP
+    result. With P = 1 the block's output equals, bit for bit, the unchanged
+    attention run on the full tensors (usp_head_attention on one head shard
+    holding every head)."""
+    w = Workload("p1", 2, 333, 0, 5, 64 if dtype == "bf16" else 48, 1, dtype, 1.0, 77, (1,))
+    q, k, v = (to_device(x, dtype) for x in make_qkv(w))
+    plan = _plan(usp, w)
+    block = usp.ulysses_attention(plan, [q], [k], [v], num_chunks=2)
+    direct = usp.head_attention(plan, [q], [k], [v])
+    torch.cuda.synchronize()
+    bits = torch.int16 if dtype == "bf16" else torch.int32
+    assert torch.equal(block[0].view(bits), direct[0].view(bits))
+    plan.close()
+
+
+def test_largest_world_and_head_count(usp):
+    """32 virtual ranks (the largest world) over 256 heads (the largest head
+    count), ragged tokens, elementwise against the oracle."""
+    w = Workload("max", 1, 97, 1, 256, 16, 32, "bf16", 1.0, 78, (1,))
+    storage, plan, out = _run_block(usp, w, 3)
+    ref = _oracle_block(w, storage, plan)
+    for r in range(plan.world):
+        assert_close(to_f64(out[r], w.dtype), ref[r], w.dtype, f"rank {r}")
+    plan.close()
+
+
+def test_fp32_largest_head_dim(usp):
+    """fp32 attention at head_dim 256, the largest the fp32 kernel is built for."""
+    w = Workload("fp32-d256", 1, 70, 0, 3, 256, 3, "fp32", 1.0, 79, (1,))
+    storage, plan, out = _run_block(usp, w, 1)
+    ref = _oracle_block(w, storage, plan)
+    for r in range(plan.world):
+        assert_close(to_f64(out[r], w.dtype), ref[r], w.dtype, f"rank {r}")
+    plan.close()
