@@ -157,30 +157,14 @@ __global__ void __launch_bounds__(32, 1) pack_tma_kernel(const __grid_constant__
 
 int encode(CUtensorMap* map, const void* base, int elem, int64_t dv, int64_t heads, int64_t rows, int64_t outer,
            int64_t head_stride, int64_t row_stride, int64_t outer_stride, int box_heads, int box_rows) {
-  typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-  static EncodeFn fn = [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeFn>(nullptr);
-    return reinterpret_cast<EncodeFn>(ptr);
-  }();
-  if (!fn) return set_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(dv), static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(head_stride), static_cast<cuuint64_t>(row_stride),
-                           static_cast<cuuint64_t>(outer_stride)};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(dv), static_cast<cuuint32_t>(box_heads),
-                       static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const uint64_t dims[4] = {static_cast<uint64_t>(dv), static_cast<uint64_t>(heads), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(outer)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(head_stride), static_cast<uint64_t>(row_stride),
+                               static_cast<uint64_t>(outer_stride)};
+  const uint32_t box[4] = {static_cast<uint32_t>(dv), static_cast<uint32_t>(box_heads),
+                           static_cast<uint32_t>(box_rows), 1};
   const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
-  CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled (pack) failed (%d)", static_cast<int>(r));
-  return USP_OK;
+  return encode_tiled_4d(map, dt, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace

@@ -209,6 +209,11 @@ inline bool fill_blocks(const AttnLaunch& L, int kv_tokens, int rows_per_tile, i
   return true;
 }
 
+// A 4-D tiled TMA map with no interleave, 256-byte L2 promotion and no
+// out-of-bounds fill, through the driver's cuTensorMapEncodeTiled.
+int encode_tiled_4d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[4],
+                    const uint64_t strides_bytes[3], const uint32_t box[4], CUtensorMapSwizzle swizzle);
+
 // 4-D TMA map (d, head, token, batch) of one 16-bit attention operand view
 // with `rows` tokens; boxes of `atom` elements x 1 head x box_rows tokens,
 // swizzled by the atom width (64: 128 B, 32: 64 B, 16: 32 B).
