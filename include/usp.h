@@ -349,6 +349,29 @@ int usp_ulysses_attention_noalloc(const usp_plan* plan, const void* const* q, co
                                   void* stream);
 
 /*
+ * usp_ulysses_attention_graph_create -- captures one usp_ulysses_attention
+ * call (its packs, attention launches and the auxiliary-stream chunk
+ * overlap) into a CUDA graph owned by the returned handle, without running it.
+ * Arguments as usp_ulysses_attention; the buffer pointers are fixed in the
+ * graph, so a caller refreshes inputs by writing into the same q/k/v buffers
+ * and replays with usp_graph_launch, one launch per block. The plan must
+ * outlive the graph only for usp_graph_destroy's bookkeeping: the graph
+ * itself holds no reference to the plan's streams or events. Errors as
+ * usp_ulysses_attention (nothing is captured then), plus USP_ERR_CUDA if the
+ * capture or instantiation fails.
+ */
+typedef struct usp_graph usp_graph;
+int usp_ulysses_attention_graph_create(usp_graph** out, const usp_plan* plan, const void* const* q,
+                                       const void* const* k, const void* const* v, void* const* o, float scale,
+                                       int32_t num_chunks, void* workspace, size_t workspace_bytes);
+
+/* Launches the captured block on `stream` (a cudaStream_t; NULL = the legacy default stream). */
+int usp_graph_launch(usp_graph* graph, void* stream);
+
+/* Releases the graph (NULL is ignored). Launches already enqueued complete normally. */
+int usp_graph_destroy(usp_graph* graph);
+
+/*
  * usp_plan_set_timing_events -- profiling hook: while set, every
  * usp_ulysses_attention call with this plan records `start` (a cudaEvent_t)
  * on its stream just before its first attention kernel and `stop` just after

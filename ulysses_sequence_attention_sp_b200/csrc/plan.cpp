@@ -828,6 +828,70 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   return USP_OK;
 }
 
+struct usp_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int device = 0;
+};
+
+int usp_ulysses_attention_graph_create(usp_graph** out, const usp_plan* plan, const void* const* q,
+                                       const void* const* k, const void* const* v, void* const* o, float scale,
+                                       int32_t num_chunks, void* workspace, size_t workspace_bytes) {
+  if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (int rc = check_plan(plan)) return rc;
+  if (int rc = device_matches(plan)) return rc;
+  NvtxRange range("usp_ulysses_attention_graph_create");
+  cudaStream_t cap = nullptr;
+  if (int rc = usp::cuda_check(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking), "cudaStreamCreate")) return rc;
+  int rc = usp::cuda_check(cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal), "cudaStreamBeginCapture");
+  cudaGraph_t graph = nullptr;
+  if (rc == USP_OK) {
+    // The call validates every argument and records only stream-ordered work.
+    const int call_rc = usp_ulysses_attention(plan, q, k, v, o, scale, num_chunks, workspace, workspace_bytes, cap);
+    const std::string call_msg = g_last_error;
+    const cudaError_t end = cudaStreamEndCapture(cap, &graph);
+    if (call_rc != USP_OK) {
+      rc = call_rc;
+      g_last_error = call_msg;
+    } else {
+      rc = usp::cuda_check(end, "cudaStreamEndCapture");
+    }
+  }
+  cudaStreamDestroy(cap);
+  if (rc != USP_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return rc;
+  }
+  usp_graph* g = new usp_graph();
+  g->graph = graph;
+  g->device = plan->device;
+  if ((rc = usp::cuda_check(cudaGraphInstantiate(&g->exec, graph, 0), "cudaGraphInstantiate")) != USP_OK) {
+    usp_graph_destroy(g);
+    return rc;
+  }
+  *out = g;
+  return USP_OK;
+}
+
+int usp_graph_launch(usp_graph* graph, void* stream) {
+  if (!graph) return usp::set_error(USP_ERR_INVALID_ARG, "graph is NULL");
+  int dev = -1;
+  if (int rc = usp::cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  if (dev != graph->device)
+    return usp::set_error(USP_ERR_INVALID_ARG, "graph was captured on device %d but device %d is current",
+                          graph->device, dev);
+  return usp::cuda_check(cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)), "cudaGraphLaunch");
+}
+
+int usp_graph_destroy(usp_graph* graph) {
+  if (!graph) return USP_OK;
+  if (graph->exec) cudaGraphExecDestroy(graph->exec);
+  if (graph->graph) cudaGraphDestroy(graph->graph);
+  delete graph;
+  return USP_OK;
+}
+
 int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode) {
   if (int rc = check_plan(plan)) return rc;
   if (mode != USP_PACK_VECTOR && mode != USP_PACK_TMA)

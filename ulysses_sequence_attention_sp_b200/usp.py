@@ -74,6 +74,11 @@ _SIGNATURES = {
                                                  ctypes.c_float, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                                  ctypes.c_void_p]),
     "usp_plan_set_pack_mode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
+    "usp_ulysses_attention_graph_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p, _c_vpp,
+                                                          _c_vpp, _c_vpp, _c_vpp, ctypes.c_float, ctypes.c_int32,
+                                                          ctypes.c_void_p, ctypes.c_size_t]),
+    "usp_graph_launch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "usp_graph_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "usp_plan_query": (ctypes.c_int, [ctypes.c_void_p, _c_i64p, _c_i64p, _c_i32p, _c_i32p]),
     "usp_scatter_sequence": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _c_vpp, ctypes.c_int64,
@@ -473,6 +478,47 @@ def ulysses_attention(plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chu
     _check(_lib.usp_ulysses_attention_lse(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), lse.data_ptr(),
                                           float(scale), num_chunks, workspace.data_ptr(), nbytes, _stream(stream)))
     return out
+
+
+class AttentionGraph:
+    """One ulysses_attention call captured into a CUDA graph owned by the
+    library; launch() replays it (one launch per block). The tensors' addresses
+    are fixed in the graph: refresh the inputs by writing into the same q/k/v
+    shards. Keeps references to every tensor it uses."""
+
+    def __init__(self, plan: Plan, q, k, v, out=None, scale: float = 0.0, num_chunks: int = 1, workspace=None):
+        shapes = [plan.seq_shard_shape(r) for r in range(plan.world)]
+        kv_shapes = [plan.kv_seq_shard_shape(r) for r in range(plan.world)]
+        out = out if out is not None else [torch.empty(s, dtype=plan.torch_dtype, device="cuda") for s in shapes]
+        for name, ts, sh in (("q", q, shapes), ("k", k, kv_shapes), ("v", v, kv_shapes), ("out", out, shapes)):
+            _check_tensors(plan, ts, sh, name)
+        need = plan.workspace_bytes(num_chunks)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+        if workspace.numel() * workspace.element_size() < need:
+            raise UspError(USP_ERR_SHAPE, f"workspace needs {need} bytes")
+        handle = ctypes.c_void_p()
+        _check(_lib.usp_ulysses_attention_graph_create(ctypes.byref(handle), plan.handle, _ptrs(q), _ptrs(k), _ptrs(v),
+                                                       _ptrs(out), float(scale), num_chunks, workspace.data_ptr(),
+                                                       workspace.numel() * workspace.element_size()))
+        self._h = handle
+        self._keep = (plan, list(q), list(k), list(v), workspace)
+        self.out = out
+
+    def launch(self, stream=None):
+        _check(_lib.usp_graph_launch(self._h, _stream(stream)))
+        return self.out
+
+    def close(self) -> None:
+        if self._h:
+            _lib.usp_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
