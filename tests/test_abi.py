@@ -112,3 +112,21 @@ def test_null_pointers_rejected(usp):
     assert b"plan is NULL" in lib.usp_last_error_message()
     lib.usp_debug_wait_timeout.restype = ctypes.c_int
     assert lib.usp_debug_wait_timeout(ctypes.c_uint32(0), None) == usp.USP_ERR_INVALID_ARG
+
+
+def test_header_compiles_and_links_from_c(usp, tmp_path):
+    """include/usp.h is plain C11: the C caller used by the GPU test compiles
+    with -Wall -Werror and links against the library (nothing is run here)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    libdir = os.path.dirname(usp.library_path())
+    out = tmp_path / "c_abi_block"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), "-o", str(out), os.path.join(ROOT, "tests", "c_abi_block.c"),
+                    "-L", libdir, "-lusp", "-L", os.path.join(cuda, "lib64"), "-lcudart", f"-Wl,-rpath,{libdir}"],
+                   check=True)
+    usage = subprocess.run([str(out)], capture_output=True, text=True)
+    assert usage.returncode == 2 and "usage" in usage.stderr
