@@ -167,6 +167,21 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
 #define USP_PACK_TMA 1
 int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode);
 
+/*
+ * usp_plan_set_attention_ctas -- caps the CTAs of this plan's tensor-core
+ * attention launches at max_ctas (0, the default: automatic). A launch with
+ * more (query tile, batch, head) items than its CTAs runs persistent CTAs:
+ * CTA c takes items c, c + max_ctas, ... and starts each item's loads and
+ * first Q K^T under the previous item's last key tiles. Automatic mode uses
+ * one CTA per SM when an item has at most 16 key tiles of 256 (short
+ * sequences, where a CTA's fixed costs are a large share), and one CTA per
+ * item otherwise. A cap below the SM count leaves SMs to kernels running
+ * beside the block on other streams. Results do not depend on it (each item
+ * is computed the same way). The fp32 path ignores it. Errors:
+ * USP_ERR_INVALID_ARG for max_ctas < 0.
+ */
+int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas);
+
 /* Copies the plan's Ulysses group size and ring size out (world and 1 for a plain plan); either may be NULL. */
 int usp_plan_query_hybrid(const usp_plan* plan, int32_t* ulysses_size, int32_t* ring_size);
 

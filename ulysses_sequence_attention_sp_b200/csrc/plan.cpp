@@ -619,6 +619,7 @@ int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const v
     L.head_dim = static_cast<int32_t>(D);
     L.dtype = plan->dtype;
     L.scale = resolve_scale(plan, scale);
+    L.max_ctas = plan->attn_ctas;
     for (int h = 0; h < hr; ++h) L.heads[h] = static_cast<uint16_t>(h);
     if (int rc = launch_attention(L, s)) return rc;
   }
@@ -784,6 +785,7 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   L.head_dim = static_cast<int32_t>(D);
   L.dtype = plan->dtype;
   L.scale = resolve_scale(plan, scale);
+  L.max_ctas = plan->attn_ctas;
   L.lse = lse;
   if (plan->ring > 1) {
     // Ring: query group g = key block g = token block of Ulysses group g
@@ -897,6 +899,13 @@ int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode) {
   if (mode != USP_PACK_VECTOR && mode != USP_PACK_TMA)
     return usp::set_error(USP_ERR_INVALID_ARG, "pack mode must be USP_PACK_VECTOR or USP_PACK_TMA (got %d)", mode);
   plan->pack_mode = mode;
+  return USP_OK;
+}
+
+int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas) {
+  if (int rc = check_plan(plan)) return rc;
+  if (max_ctas < 0) return usp::set_error(USP_ERR_INVALID_ARG, "attention CTA cap must be >= 0 (got %d)", max_ctas);
+  plan->attn_ctas = max_ctas;
   return USP_OK;
 }
 

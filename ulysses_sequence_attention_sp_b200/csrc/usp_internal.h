@@ -33,6 +33,7 @@ struct usp_plan {
   int32_t head_ranks = 0;
   int32_t ring = 1;
   int32_t pack_mode = 0;  // USP_PACK_VECTOR or USP_PACK_TMA: how seq->head packs move data
+  int32_t attn_ctas = 0;  // cap on the attention kernel's CTAs (0: automatic)
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
@@ -184,6 +185,7 @@ struct AttnLaunch {
   int32_t head_dim;
   int32_t dtype;
   float scale;
+  int32_t max_ctas;  // cap on the tensor-core kernel's CTAs (0: automatic)
   uint16_t heads[USP_MAX_HEADS];
 };
 

@@ -74,6 +74,7 @@ _SIGNATURES = {
                                                  ctypes.c_float, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                                  ctypes.c_void_p]),
     "usp_plan_set_pack_mode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
+    "usp_plan_set_attention_ctas": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
     "usp_ulysses_attention_graph_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p, _c_vpp,
                                                           _c_vpp, _c_vpp, _c_vpp, ctypes.c_float, ctypes.c_int32,
                                                           ctypes.c_void_p, ctypes.c_size_t]),
@@ -267,6 +268,12 @@ class Plan:
             raise UspError(USP_ERR_INVALID_ARG, f"pack mode must be one of {sorted(codes)}")
         _check(_lib.usp_plan_set_pack_mode(self.handle, codes[mode]))
         self.pack_mode = mode
+
+    def set_attention_ctas(self, max_ctas: int) -> None:
+        """Caps the tensor-core attention kernel's CTAs (0: automatic); with
+        fewer CTAs than (query tile, batch, head) items each CTA walks several."""
+        _check(_lib.usp_plan_set_attention_ctas(self.handle, int(max_ctas)))
+        self.attention_ctas = int(max_ctas)
 
     def workspace_bytes(self, num_chunks: int = 1) -> int:
         n = ctypes.c_size_t()
