@@ -388,24 +388,39 @@ static int scatter_gather(const usp_plan* plan, int dir, const void* full, void*
   if (row_bytes == 0) row_bytes = static_cast<int64_t>(plan->heads) * plan->head_dim * plan->elem;
   if (outer < 1 || row_bytes < 1) return usp::set_error(USP_ERR_SHAPE, "outer and row_bytes must be positive");
   if (row_bytes % 16 != 0) return usp::set_error(USP_ERR_ALIGN, "row_bytes must be a multiple of 16");
-  usp::PermuteArgs a;
+  // Every rank's token window is one contiguous run of rows per batch element
+  // in both buffers; the prefix rows go to every shard (scatter) or come from
+  // rank 0's (gather).
+  usp::CopyArgs a;
   memset(&a, 0, sizeof(a));
-  a.dir = dir;
-  fill_seq_side(a, plan, outer);
-  a.n_head = 1;
-  a.ntensors = 1;
-  a.heads = 1;
-  a.dv = static_cast<int32_t>(row_bytes / 16);
-  a.head_layout = 0;
-  a.full_tokens = plan->tokens();
-  a.head_start[0] = 0;
-  a.head_start[1] = 1;
-  a.nsel = 1;
-  a.sel_head[0] = 0;
-  a.sel_rank[0] = 0;
-  a.head_ptr[0][0] = const_cast<void*>(full);
-  for (int r = 0; r < plan->world; ++r) a.seq_ptr[0][r] = shards[r];
-  return usp::launch_permute(a, 16, stream);
+  a.to_shards = dir;
+  a.outer = outer;
+  a.nv = row_bytes / 16;
+  a.full_rows = plan->tokens();
+  a.full = const_cast<void*>(full);
+  const int64_t pre = plan->prefix;
+  int n = 0;
+  for (int r = 0; r < plan->world; ++r) {
+    a.shards[r] = shards[r];
+    a.shard[n] = r;
+    a.shard_rows[n] = pre + plan->tok_len[r];
+    a.srow0[n] = pre;
+    a.frow0[n] = pre + plan->tok_start[r];
+    a.rows[n] = plan->tok_len[r];
+    ++n;
+  }
+  if (pre > 0) {
+    for (int r = 0; r < (dir == 1 ? plan->world : 1); ++r) {
+      a.shard[n] = r;
+      a.shard_rows[n] = pre + plan->tok_len[r];
+      a.srow0[n] = 0;
+      a.frow0[n] = 0;
+      a.rows[n] = pre;
+      ++n;
+    }
+  }
+  a.nkinds = n;
+  return usp::launch_copy_rows(a, stream);
 }
 
 int usp_scatter_sequence(const usp_plan* plan, const void* x_full, void* const* x_shards, int64_t outer,

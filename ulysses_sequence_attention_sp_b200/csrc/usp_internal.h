@@ -120,6 +120,32 @@ struct RowsArgs {
 };
 
 int launch_all_gather_rows(const RowsArgs& a, int vec_bytes, cudaStream_t stream);
+
+// ------------------------------------------------- segmented row copy
+// scatter_sequence / gather_sequence: every kind s of segment is a run of
+// rows[s] rows that is contiguous, within each of the `outer` batch elements,
+// in both buffers: rows [srow0[s], +rows[s]) of shard `shard[s]`, laid out
+// [outer][shard_rows[s]][nv], and rows [frow0[s], +rows[s]) of the full buffer
+// [outer][full_rows][nv]. nv counts 16-byte vectors per row.
+constexpr int kMaxCopyKinds = 2 * USP_MAX_WORLD;  // every rank's token window + the prefix rows
+struct CopyArgs {
+  int32_t to_shards;  // 1: full -> shards (scatter), 0: shards -> full (gather)
+  int32_t nkinds;
+  int64_t outer;
+  int64_t nv;
+  int64_t full_rows;
+  int32_t shard[kMaxCopyKinds];
+  int64_t shard_rows[kMaxCopyKinds];
+  int64_t srow0[kMaxCopyKinds];
+  int64_t frow0[kMaxCopyKinds];
+  int64_t rows[kMaxCopyKinds];
+  int64_t seg_tiles[kMaxCopyKinds];        // set by the launcher
+  int64_t tile_prefix[kMaxCopyKinds + 1];  // set by the launcher
+  void* full;
+  void* shards[USP_MAX_WORLD];
+};
+
+int launch_copy_rows(const CopyArgs& a, cudaStream_t stream);
 int launch_reduce_scatter_rows(const RowsArgs& a, int vec_bytes, int dtype, cudaStream_t stream);
 
 // -------------------------------------------------------------- attention
