@@ -155,11 +155,11 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
 /*
  * usp_plan_set_pack_mode -- how this plan's sequence -> head moves
  * (usp_ulysses_seq_to_head(_kv) and the pack inside usp_ulysses_attention)
- * run. USP_PACK_VECTOR (the default): 16-byte vector loads and stores, one
- * warp per sequence row. USP_PACK_TMA: TMA tile copies, global -> shared ->
- * global, one head unit of up to 64 rows per tile, no multicast; used where a
- * head unit (head_dim * element size) is a multiple of 16 bytes of at most
- * 256 elements, the vector kernel otherwise. Both give identical bytes
+ * run. USP_PACK_TMA (the default): TMA tile copies, global -> shared ->
+ * global, up to 64 rows of a few head units per tile, no multicast; used
+ * where a head unit (head_dim * element size) is a multiple of 16 bytes of at
+ * most 256 elements, the vector kernel otherwise. USP_PACK_VECTOR: 16-byte
+ * vector loads and stores, one warp per segment of a sequence row. Both give identical bytes
  * ("h3_blackwell_runtime/distributed.py", seq_to_heads). Errors:
  * USP_ERR_INVALID_ARG for an unknown mode.
  */

@@ -32,7 +32,7 @@ struct usp_plan {
   // consecutive ranks. The plain block is head_ranks == world, ring == 1.
   int32_t head_ranks = 0;
   int32_t ring = 1;
-  int32_t pack_mode = 0;  // USP_PACK_VECTOR or USP_PACK_TMA: how seq->head packs move data
+  int32_t pack_mode = USP_PACK_TMA;  // USP_PACK_TMA (default) or USP_PACK_VECTOR: how seq->head packs move data
   int32_t attn_ctas = 0;  // cap on the attention kernel's CTAs (0: automatic)
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs

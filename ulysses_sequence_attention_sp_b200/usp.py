@@ -202,6 +202,7 @@ class Plan:
         self.kv_heads = kv_heads
         self.ulysses_size = world // ring_size
         self.ring_size = ring_size
+        self.pack_mode = "tma"
         self.batch, self.seq_len, self.heads, self.head_dim = batch, seq_len, heads, head_dim
         self.world, self.dtype_code, self.prefix = world, code, prefix
         self.torch_dtype = _TORCH[code]
@@ -262,7 +263,7 @@ class Plan:
         return t
 
     def set_pack_mode(self, mode: str) -> None:
-        """'vector' (default) or 'tma': how sequence -> head moves run (same bytes)."""
+        """'tma' (default) or 'vector': how sequence -> head moves run (same bytes)."""
         codes = {"vector": 0, "tma": 1}
         if mode not in codes:
             raise UspError(USP_ERR_INVALID_ARG, f"pack mode must be one of {sorted(codes)}")
