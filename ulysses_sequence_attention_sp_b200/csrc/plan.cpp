@@ -140,8 +140,10 @@ void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) 
 
 // A sequence -> head move: TMA tile copies when the plan asks for them and the
 // head unit allows it (a multiple of 16 bytes), else 16-byte vector copies.
+// (The TMA launcher counts rows in 32 bits.)
 int launch_pack(const usp_plan* plan, const usp::PermuteArgs& a, int vec, int64_t unit, cudaStream_t stream) {
-  if (a.dir == 0 && plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit))
+  if (a.dir == 0 && plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit) &&
+      a.seq_rows[a.n_seq] <= INT32_MAX)
     return usp::launch_pack_tma(a, plan->elem, unit, stream);
   return usp::launch_permute(a, vec, stream);
 }
@@ -471,7 +473,8 @@ static int head_slice_gather(const usp_plan* plan, int dir, const void* full, vo
   select_all_heads(a, plan->heads, plan->head_start, plan->world);
   a.seq_ptr[0][0] = const_cast<void*>(full);
   for (int r = 0; r < plan->world; ++r) a.head_ptr[0][r] = shards[r];
-  return usp::launch_permute(a, vec, stream);
+  // The slice is a sequence -> head move (one sequence-side buffer holding every row).
+  return dir == 0 ? launch_pack(plan, a, vec, unit, stream) : usp::launch_permute(a, vec, stream);
 }
 
 int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards, int64_t rows,
