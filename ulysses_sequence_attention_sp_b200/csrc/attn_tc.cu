@@ -915,6 +915,102 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_persistent_kernel(const _
     uint64_t* xbar = &bars->xbar[quarter];
     const float sl2 = p.scale_log2;
     bool ok = true;
+    // Epilogue of item e_it (running maximum e_m, combined denominator e_l):
+    // O is read from TMEM, normalised and stored to its rows' sequence shards,
+    // and o_empty lets the next item's first P V overwrite O.
+    auto epilogue = [&](int e_it, float e_m, float e_l) {
+      tc_fence_after();
+      const Item I = decode_item<RING>(p, first_item + e_it * item_stride);
+      const float inv_l = 1.f / e_l;
+      const int t = I.row0 + row;
+      bool row_ok = t < T;
+      if constexpr (RING) row_ok = t < p.q_start[I.g + 1] && t < T;
+      const int b = I.b, hm = I.hm;
+      if (p.lse != nullptr && part == 0 && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
+        const int64_t li = (static_cast<int64_t>(hm) * p.batch + b) * T + t;
+        if (in_bounds(li, 1, p.lse_ext, 22, &g_attn_bounds)) p.lse[li] = (e_m + log2f(e_l)) * 0.69314718055994531f;
+      }
+      const AttnOut& out = p.out;
+      // Destination(s) of this row.
+      int seg_lo = 0, seg_hi = 0;
+      int64_t row_in_seg = 0;
+      if (row_ok) {
+        if (t < out.prefix) {
+          seg_lo = 0;
+          seg_hi = out.nseg;
+          row_in_seg = t;
+        } else {
+          const int64_t tok = t - out.prefix;
+          int sg = 0;
+          while (sg + 1 < out.nseg && tok >= out.seg_start[sg + 1]) ++sg;
+          seg_lo = sg;
+          seg_hi = sg + 1;
+          row_in_seg = out.prefix + tok - out.seg_start[sg];
+        }
+      }
+      // A warp holds 32 rows x 16 columns of each O chunk (32 bytes a row).
+      // Lanes are paired per row for the stores: in round h, lane t writes
+      // half t & 1 of row 16h + t/2 of the warp, so each store instruction
+      // fills 16 whole 32-byte sectors instead of touching 32 half sectors.
+      // Every softmax thread arrives on o_empty once it has read its last
+      // chunk of O, or at once if its part holds none (head_dim < 64).
+      if (part >= kOChunks) {
+        tc_fence_before();
+        mbar_arrive(&bars->o_empty);
+      }
+      for (int c = part; c < kOChunks; c += kParts) {
+        uint32_t o[16];
+        tmem_ld16(lane_addr + kColO + c * 16, o);
+        tmem_wait_ld();
+        if (c + kParts >= kOChunks) {  // this thread's last chunk: O is free for the next item
+          tc_fence_before();
+          mbar_arrive(&bars->o_empty);
+        }
+        uint4 w0, w1;
+        w0.x = pack2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l, BF16);
+        w0.y = pack2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l, BF16);
+        w0.z = pack2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l, BF16);
+        w0.w = pack2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l, BF16);
+        w1.x = pack2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l, BF16);
+        w1.y = pack2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l, BF16);
+        w1.z = pack2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l, BF16);
+        w1.w = pack2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l, BF16);
+        const bool hi_half = lane & 1;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // Row src's two halves come from lane src (which holds that row);
+          // this lane keeps the half it writes.
+          const int src = 16 * h + (lane >> 1);
+          uint4 a, v;
+          a.x = __shfl_sync(0xffffffffu, w0.x, src);
+          a.y = __shfl_sync(0xffffffffu, w0.y, src);
+          a.z = __shfl_sync(0xffffffffu, w0.z, src);
+          a.w = __shfl_sync(0xffffffffu, w0.w, src);
+          v.x = __shfl_sync(0xffffffffu, w1.x, src);
+          v.y = __shfl_sync(0xffffffffu, w1.y, src);
+          v.z = __shfl_sync(0xffffffffu, w1.z, src);
+          v.w = __shfl_sync(0xffffffffu, w1.w, src);
+          const uint4 val = hi_half ? v : a;
+          const int lo = __shfl_sync(0xffffffffu, seg_lo, src);
+          const int hi = __shfl_sync(0xffffffffu, seg_hi, src);
+          const int64_t r_in = __shfl_sync(0xffffffffu, row_in_seg, src);
+          for (int sg = lo; sg < hi; ++sg) {
+            const int64_t rows_s = out.prefix + out.seg_len[sg];
+            const int64_t elem =
+                ((static_cast<int64_t>(b) * rows_s + r_in) * out.out_heads + hm) * D + c * 16 + (lane & 1) * 8;
+            if (!in_bounds(elem, 8, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 21, &g_attn_bounds))
+              continue;
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem) = val;
+          }
+        }
+      }
+      if (threadIdx.x == 0) USP_TRACE_EV(12, e_it);
+    };
+    // An item's epilogue is deferred to the first tile of the next item: that
+    // tile's softmax runs while the item's last P V completes, and its P is
+    // stored (so the next P V, which overwrites O, can start) right after.
+    float m_prev = 0.f, l_prev = 1.f;
+    int last_it = -1;
     // jg = jg0 + j counts key tiles over the CTA's items: the phase of s_full,
     // p_full and pv_done. The quarter's exchange barrier completes once per
     // tile and once per item (the denominator combine), so its phase is jg + it.
@@ -1030,6 +1126,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_persistent_kernel(const _
         if (threadIdx.x == 0) USP_TRACE_EV(8, jg);
         // P is single-buffered: it was last read by the previous tile's P V.
         if (jg >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (jg - 1) & 1, abort_flag, &g_attn_error, 32, kWaitLimitNs))) { ok = false; break; }
+        if (j == 0 && it > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full, (it - 1) & 1, abort_flag, &g_attn_error, 33, kWaitLimitNs))) { ok = false; break; }
+          if (threadIdx.x == 0) USP_TRACE_EV(11, it - 1);
+          epilogue(it - 1, m_prev, l_prev);
+        }
         tc_fence_after();
         tmem_st32(lane_addr + kColP + part * (kCols / 2), pk);
         tmem_wait_st();
@@ -1054,96 +1155,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_persistent_kernel(const _
         if (threadIdx.x == 0) USP_TRACE_EV(10, it);
         if (ok) l = (xrow[0] + xrow[kBM]) + (xrow[2 * kBM] + xrow[3 * kBM]);
       }
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_full, it & 1, abort_flag, &g_attn_error, 33, kWaitLimitNs));
-      if (threadIdx.x == 0) USP_TRACE_EV(11, it);
-      if (ok) {
-        tc_fence_after();
-        const Item I = decode_item<RING>(p, first_item + it * item_stride);
-        const float inv_l = 1.f / l;
-        const int t = I.row0 + row;
-        bool row_ok = t < T;
-        if constexpr (RING) row_ok = t < p.q_start[I.g + 1] && t < T;
-        const int b = I.b, hm = I.hm;
-        if (p.lse != nullptr && part == 0 && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
-          const int64_t li = (static_cast<int64_t>(hm) * p.batch + b) * T + t;
-          if (in_bounds(li, 1, p.lse_ext, 22, &g_attn_bounds)) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
-        }
-        const AttnOut& out = p.out;
-        // Destination(s) of this row.
-        int seg_lo = 0, seg_hi = 0;
-        int64_t row_in_seg = 0;
-        if (row_ok) {
-          if (t < out.prefix) {
-            seg_lo = 0;
-            seg_hi = out.nseg;
-            row_in_seg = t;
-          } else {
-            const int64_t tok = t - out.prefix;
-            int sg = 0;
-            while (sg + 1 < out.nseg && tok >= out.seg_start[sg + 1]) ++sg;
-            seg_lo = sg;
-            seg_hi = sg + 1;
-            row_in_seg = out.prefix + tok - out.seg_start[sg];
-          }
-        }
-        // A warp holds 32 rows x 16 columns of each O chunk (32 bytes a row).
-        // Lanes are paired per row for the stores: in round h, lane t writes
-        // half t & 1 of row 16h + t/2 of the warp, so each store instruction
-        // fills 16 whole 32-byte sectors instead of touching 32 half sectors.
-        // Every softmax thread arrives on o_empty once it has read its last
-        // chunk of O, or at once if its part holds none (head_dim < 64).
-        if (part >= kOChunks) {
-          tc_fence_before();
-          mbar_arrive(&bars->o_empty);
-        }
-        for (int c = part; c < kOChunks; c += kParts) {
-          uint32_t o[16];
-          tmem_ld16(lane_addr + kColO + c * 16, o);
-          tmem_wait_ld();
-          if (c + kParts >= kOChunks) {  // this thread's last chunk: O is free for the next item
-            tc_fence_before();
-            mbar_arrive(&bars->o_empty);
-          }
-          uint4 w0, w1;
-          w0.x = pack2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l, BF16);
-          w0.y = pack2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l, BF16);
-          w0.z = pack2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l, BF16);
-          w0.w = pack2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l, BF16);
-          w1.x = pack2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l, BF16);
-          w1.y = pack2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l, BF16);
-          w1.z = pack2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l, BF16);
-          w1.w = pack2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l, BF16);
-          const bool hi_half = lane & 1;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // Row src's two halves come from lane src (which holds that row);
-            // this lane keeps the half it writes.
-            const int src = 16 * h + (lane >> 1);
-            uint4 a, v;
-            a.x = __shfl_sync(0xffffffffu, w0.x, src);
-            a.y = __shfl_sync(0xffffffffu, w0.y, src);
-            a.z = __shfl_sync(0xffffffffu, w0.z, src);
-            a.w = __shfl_sync(0xffffffffu, w0.w, src);
-            v.x = __shfl_sync(0xffffffffu, w1.x, src);
-            v.y = __shfl_sync(0xffffffffu, w1.y, src);
-            v.z = __shfl_sync(0xffffffffu, w1.z, src);
-            v.w = __shfl_sync(0xffffffffu, w1.w, src);
-            const uint4 val = hi_half ? v : a;
-            const int lo = __shfl_sync(0xffffffffu, seg_lo, src);
-            const int hi = __shfl_sync(0xffffffffu, seg_hi, src);
-            const int64_t r_in = __shfl_sync(0xffffffffu, row_in_seg, src);
-            for (int sg = lo; sg < hi; ++sg) {
-              const int64_t rows_s = out.prefix + out.seg_len[sg];
-              const int64_t elem =
-                  ((static_cast<int64_t>(b) * rows_s + r_in) * out.out_heads + hm) * D + c * 16 + (lane & 1) * 8;
-              if (!in_bounds(elem, 8, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 21, &g_attn_bounds))
-                continue;
-              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem) = val;
-            }
-          }
-        }
-        if (threadIdx.x == 0) USP_TRACE_EV(12, it);
-      }
+      m_prev = m;
+      l_prev = l;
+      last_it = it;
+    }
+    // The last item's epilogue.
+    if (ok && last_it >= 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&bars->o_full, last_it & 1, abort_flag, &g_attn_error, 33, kWaitLimitNs))) {
+      if (threadIdx.x == 0) USP_TRACE_EV(11, last_it);
+      epilogue(last_it, m_prev, l_prev);
     }
   }
 
