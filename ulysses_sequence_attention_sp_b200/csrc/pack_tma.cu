@@ -1,7 +1,10 @@
 // TMA-staged seq->head pack ("h3_blackwell_runtime/distributed.py -- Ragged
-// Ulysses sequence-parallel transport", SequenceParallelContext.seq_to_heads):
-// the same permutation as permute_kernel with dir = 0, moved by the Tensor
-// Memory Accelerator instead of vector loads and stores.
+// Ulysses sequence-parallel transport", SequenceParallelContext.seq_to_heads),
+// and the same move backwards (heads_to_seq): the permutation of
+// permute_kernel, moved by the Tensor Memory Accelerator instead of vector
+// loads and stores. Backwards, each unit's box is loaded from the head shard
+// and stored to the sequence shard; the replicated prefix rows land in rank
+// 0's shard only (the caller copies them to the others).
 //
 // A work unit is one head unit (D elements) of n consecutive token rows of one
 // source rank: a 4-D tile load (d, head, row, batch) of box (D, 1, n, 1) from
@@ -43,10 +46,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: only a broken copy wai
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 struct PackTmaParams {
-  CUtensorMap src[3][USP_MAX_WORLD];
-  CUtensorMap dst[3][USP_MAX_WORLD];
+  CUtensorMap src[3][USP_MAX_WORLD];     // sequence-side buffers
+  CUtensorMap dst[3][USP_MAX_WORLD];     // head-side buffers
   int64_t total_units;
   int32_t ntensors, n_seq, nsel, outer;
+  int32_t dir;                           // 0: sequence -> head; 1: head -> sequence (same units, boxes swapped)
   int32_t hb;                            // head units per tile (divides every buffer's selected count)
   int32_t ngroups;                       // nsel / hb
   int32_t rows;                          // n
@@ -125,8 +129,11 @@ __global__ void __launch_bounds__(32, 1) pack_tma_kernel(const __grid_constant__
     in_bounds(u.row, p.rows, p.r0[u.s] + p.cnt[u.s], 61, &g_pack_bounds);
     in_bounds(p.sel_head[u.i], p.hb, p.heads, 62, &g_pack_bounds);
     mbar_arrive_expect_tx(&full[st], p.box_bytes);
-    tma_load_4d(&p.src[u.t][u.s], &full[st], smem + static_cast<size_t>(st) * p.stage_bytes, 0, p.sel_head[u.i],
-                u.row, u.b);
+    uint8_t* stage = smem + static_cast<size_t>(st) * p.stage_bytes;
+    if (p.dir == 0)
+      tma_load_4d(&p.src[u.t][u.s], &full[st], stage, 0, p.sel_head[u.i], u.row, u.b);
+    else
+      tma_load_4d(&p.dst[u.t][p.sel_rank[u.i]], &full[st], stage, 0, p.sel_local[u.i], u.tok, u.b);
   };
   const int64_t pro = mine < kStages - 1 ? mine : kStages - 1;
   for (int64_t k = 0; k < pro; ++k) load(k);
@@ -143,8 +150,11 @@ __global__ void __launch_bounds__(32, 1) pack_tma_kernel(const __grid_constant__
         !in_bounds(u.tok, p.rows, p.full_tokens, 65, &g_pack_bounds)) {
       bulk_commit_group();  // an empty group keeps the stage accounting of wait_group.read
     } else {
-      tma_store_4d(&p.dst[u.t][p.sel_rank[u.i]], smem + static_cast<size_t>(st) * p.stage_bytes, 0,
-                   p.sel_local[u.i], u.tok, u.b);
+      uint8_t* stage = smem + static_cast<size_t>(st) * p.stage_bytes;
+      if (p.dir == 0)
+        tma_store_4d(&p.dst[u.t][p.sel_rank[u.i]], stage, 0, p.sel_local[u.i], u.tok, u.b);
+      else
+        tma_store_4d(&p.src[u.t][u.s], stage, 0, p.sel_head[u.i], u.row, u.b);
       bulk_commit_group();
     }
     if (issued < mine) {
@@ -180,7 +190,7 @@ bool pack_tma_supported(int elem, int64_t unit_bytes) {
 }
 
 int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStream_t stream) {
-  if (a.dir != 0) return set_error(USP_ERR_INVALID_ARG, "internal: the TMA pack only moves sequence -> head");
+  if (a.dir != 0 && a.dir != 1) return set_error(USP_ERR_INVALID_ARG, "internal: bad direction %d", a.dir);
   if (a.nsel == 0 || a.seq_rows[a.n_seq] == 0) return USP_OK;
   const int64_t dv = unit_bytes / elem;
   if (!pack_tma_supported(elem, unit_bytes))
@@ -188,6 +198,7 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
   thread_local PackTmaParams p;  // ~25 KB: built on the host, copied into the launch's parameters
   memset(&p, 0, sizeof(p));
   p.ntensors = a.ntensors;
+  p.dir = a.dir;
   p.n_seq = a.n_seq;
   p.nsel = a.nsel;
   p.outer = static_cast<int32_t>(a.outer);

@@ -138,14 +138,38 @@ void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) 
     }
 }
 
-// A sequence -> head move: TMA tile copies when the plan asks for them and the
+// A sequence <-> head move: TMA tile copies when the plan asks for them and the
 // head unit allows it (a multiple of 16 bytes), else 16-byte vector copies.
-// (The TMA launcher counts rows in 32 bits.)
+// (The TMA launcher counts rows in 32 bits.) Head -> sequence by TMA needs
+// every head selected: the replicated prefix rows are then copied whole from
+// rank 0's shard to the others.
 int launch_pack(const usp_plan* plan, const usp::PermuteArgs& a, int vec, int64_t unit, cudaStream_t stream) {
-  if (a.dir == 0 && plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit) &&
-      a.seq_rows[a.n_seq] <= INT32_MAX)
-    return usp::launch_pack_tma(a, plan->elem, unit, stream);
-  return usp::launch_permute(a, vec, stream);
+  const bool tma = plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit) &&
+                   a.seq_rows[a.n_seq] <= INT32_MAX && (a.dir == 0 || a.nsel == a.heads);
+  if (!tma) return usp::launch_permute(a, vec, stream);
+  if (int rc = usp::launch_pack_tma(a, plan->elem, unit, stream)) return rc;
+  if (a.dir == 0 || a.prefix == 0 || a.n_seq < 2) return USP_OK;
+  for (int t = 0; t < a.ntensors; ++t) {
+    usp::CopyArgs c;
+    memset(&c, 0, sizeof(c));
+    c.to_shards = 1;
+    c.outer = a.outer;
+    c.nv = a.heads * unit / 16;
+    c.full_rows = a.prefix + a.tok_len[0];
+    c.full = a.seq_ptr[t][0];
+    for (int s = 1; s < a.n_seq; ++s) {
+      const int k = s - 1;
+      c.shards[s] = a.seq_ptr[t][s];
+      c.shard[k] = s;
+      c.shard_rows[k] = a.prefix + a.tok_len[s];
+      c.srow0[k] = 0;
+      c.frow0[k] = 0;
+      c.rows[k] = a.prefix;
+    }
+    c.nkinds = a.n_seq - 1;
+    if (int rc = usp::launch_copy_rows(c, stream)) return rc;
+  }
+  return USP_OK;
 }
 
 // kv selects the k/v head geometry (Hkv heads split by kv_head_start) instead
@@ -473,8 +497,9 @@ static int head_slice_gather(const usp_plan* plan, int dir, const void* full, vo
   select_all_heads(a, plan->heads, plan->head_start, plan->world);
   a.seq_ptr[0][0] = const_cast<void*>(full);
   for (int r = 0; r < plan->world; ++r) a.head_ptr[0][r] = shards[r];
-  // The slice is a sequence -> head move (one sequence-side buffer holding every row).
-  return dir == 0 ? launch_pack(plan, a, vec, unit, stream) : usp::launch_permute(a, vec, stream);
+  // The slice is a sequence -> head move and the gather its inverse (one
+  // sequence-side buffer holding every row).
+  return launch_pack(plan, a, vec, unit, stream);
 }
 
 int usp_sp_head_slice(const usp_plan* plan, const void* x_full, void* const* x_head_shards, int64_t rows,
