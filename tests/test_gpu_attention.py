@@ -188,6 +188,31 @@ def test_full_size_sampled_rows(usp, w):
     plan.close()
 
 
+@pytest.mark.parametrize("w", [VIDEO, CHUNKED], ids=lambda w: w.name)
+def test_full_size_every_row_against_fp32_kernel(usp, w):
+    """Secondary signal at full size: every output element of the tensor-core
+    block against the fp32 CUDA-core kernel run on the same values (the bf16
+    inputs upcast exactly), with the bf16 tolerances. The float64 oracle
+    checks sampled rows of the same workloads above."""
+    storage, plan, out = _run_block(usp, w, w.num_chunks[0])
+    plan32 = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, "fp32", w.prefix)
+    shards32 = [usp.scatter_sequence(plan32, torch.from_numpy(bf16_bits_to_f32(x)).cuda()) for x in storage]
+    del storage
+    out32 = usp.ulysses_attention(plan32, *shards32)
+    torch.cuda.synchronize()
+    assert usp.device_status() == 0
+    for r in range(w.world):
+        got = out[r].double()
+        ref = out32[r].double()
+        diff = (got - ref).abs()
+        st = {"max_abs": diff.max().item(), "mean_abs": diff.mean().item(),
+              "rel_l2": ((got - ref).norm() / ref.norm()).item(), "nan": int(torch.isnan(got).sum().item())}
+        assert st["nan"] == 0 and st["max_abs"] <= 2e-2 and st["mean_abs"] <= 2e-3 and st["rel_l2"] <= 1e-2, (r, st)
+    print(w.name, "rank", w.world - 1, st)
+    plan.close()
+    plan32.close()
+
+
 def test_vit_full_elementwise(usp):
     """The ViT workload is small enough for the full float64 oracle."""
     storage, plan, out = _run_block(usp, VIT, 1)
