@@ -95,10 +95,6 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units
 #define USP_PERSIST_MAX_TILES 16
 #endif
 constexpr int kPersistMaxTiles = USP_PERSIST_MAX_TILES;  // key tiles per item up to which CTAs are persistent
-#ifndef USP_POLY_EVERY
-#define USP_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = USP_POLY_EVERY;         // 0: every exp2 on MUFU
 
 template <int D>
 struct Cfg {
@@ -514,23 +510,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       uint32_t pk[kCols / 2];
       float psum;
       {
-        // Scalar FFMA / MUFU / FADD per element. Built with USP_POLY_EVERY=n > 0,
-        // on full parts one pair in n goes through the FMA-pipe polynomial
-        // instead of MUFU (measured no faster here, so off by default).
+        // One FFMA, one MUFU exp2 and one FADD per element. Full parts and
+        // parts with masked columns take separate (identical) loops: the
+        // split lets the compiler allocate the loop without a spill.
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         const float negm = -m;
         if (valid >= kCols) {
 #pragma unroll
           for (int c = 0; c < kCols; c += 2) {
-            const float x0 = fmaf(s[c], sl2, negm);
-            const float x1 = fmaf(s[c + 1], sl2, negm);
-            float p0, p1;
-            if (kPolyEvery > 0 && (c / 2) % kPolyEvery == kPolyEvery - 1) {
-              f2_unpack(exp2_poly_f2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            const float p0 = ex2_approx(fmaf(s[c], sl2, negm));
+            const float p1 = ex2_approx(fmaf(s[c + 1], sl2, negm));
             acc[c & 7] += p0;
             acc[(c + 1) & 7] += p1;
             pk[c / 2] = pack2(p0, p1, BF16);
@@ -1089,23 +1078,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_persistent_kernel(const _
         uint32_t pk[kCols / 2];
         float psum;
         {
-          // Scalar FFMA / MUFU / FADD per element. Built with USP_POLY_EVERY=n > 0,
-          // on full parts one pair in n goes through the FMA-pipe polynomial
-          // instead of MUFU (measured no faster here, so off by default).
+          // One FFMA, one MUFU exp2 and one FADD per element. Full parts and
+          // parts with masked columns take separate (identical) loops: the
+          // split lets the compiler allocate the loop without a spill.
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           const float negm = -m;
           if (valid >= kCols) {
   #pragma unroll
             for (int c = 0; c < kCols; c += 2) {
-              const float x0 = fmaf(s[c], sl2, negm);
-              const float x1 = fmaf(s[c + 1], sl2, negm);
-              float p0, p1;
-              if (kPolyEvery > 0 && (c / 2) % kPolyEvery == kPolyEvery - 1) {
-                f2_unpack(exp2_poly_f2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f))), p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
+              const float p0 = ex2_approx(fmaf(s[c], sl2, negm));
+              const float p1 = ex2_approx(fmaf(s[c + 1], sl2, negm));
               acc[c & 7] += p0;
               acc[(c + 1) & 7] += p1;
               pk[c / 2] = pack2(p0, p1, BF16);

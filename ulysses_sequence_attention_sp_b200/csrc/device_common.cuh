@@ -32,24 +32,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// try_wait. Built with USP_SUSPEND_HINT_NS > 0, it passes that suspend-time
-// hint so a thread whose phase is not complete is suspended in hardware (up to
-// the hint) instead of returning at once; the default form leaves the
-// suspension time to the hardware.
-#ifndef USP_SUSPEND_HINT_NS
-#define USP_SUSPEND_HINT_NS 0
-#endif
+// try_wait: returns once the phase completes or the hardware's suspend time runs out.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-#if USP_SUSPEND_HINT_NS > 0
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(USP_SUSPEND_HINT_NS))
-      : "memory");
-#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -57,7 +42,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
-#endif
   return ok != 0;
 }
 
@@ -256,30 +240,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// 2^x for a pair of floats on the FMA pipe (no MUFU), x >= -125 and x < 2^22:
-// n = round(x) via the 1.5*2^23 rounding constant, f = x - n in [-1/2, 1/2],
-// 2^f by a degree-3 polynomial (Remez fit of the relative error, max 7.5e-5;
-// coefficients from csrc/fit_exp2_poly.py), and 2^n added to the exponent
-// field as an integer. Cody and Waite's argument reduction.
-__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t round2 = f2_pack(kRound, kRound);
-  const uint64_t neg_round2 = f2_pack(-kRound, -kRound);
-  const uint64_t t = f2_add(x, round2);            // low mantissa bits hold round(x)
-  const uint64_t n = f2_add(t, neg_round2);        // round(x) as float
-  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);  // x - n, exact
-  uint64_t p = f2_fma(f, f2_pack(0.055171669f, 0.055171669f), f2_pack(0.24261112f, 0.24261112f));
-  p = f2_fma(p, f, f2_pack(0.69326099f, 0.69326099f));
-  p = f2_fma(p, f, f2_pack(0.99992807f, 0.99992807f));
-  float t0, t1, p0, p1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(p, p0, p1);
-  // exponent(p) += round(x): the integer in t's low bits, shifted to bit 23
-  const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);
-  const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
-  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
 }
 
 // Packs two floats into bf16x2 / f16x2 with round-to-nearest-even; `lo` in bits 0-15.
