@@ -66,6 +66,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-reshard", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (measured after the headline, 1 GPU only)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying the step as one CUDA graph")
     return ap.parse_args()
@@ -258,6 +260,194 @@ def workload_config(w, num_chunks, n_gpus):
 
 
 # ---------------------------------------------------------------- our arm
+class BlockBench:
+    """One workload's step on this device: scatter_sequence of q, k and v into
+    the virtual-rank shards, ulysses_attention (pack, attention, fused
+    head->seq) and gather_sequence of the output.
+
+    The step's calls are stream-ordered and synchronise nothing, so each timed
+    step is captured as a CUDA graph (one graph per step, each with its own
+    pair of events around the attention kernels), which removes the Python
+    launch cost that dominates the small workloads. Workloads whose q/k/v fit
+    in L2 get a 512 MiB write between timed steps, whose time is measured apart
+    and subtracted."""
+
+    def __init__(self, usp, torch, dev, w, n_chunks, steps, seed, graph=True):
+        self.usp, self.torch, self.dev, self.w, self.n_chunks, self.steps = usp, torch, dev, w, n_chunks, steps
+        self.plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix,
+                             kv_heads=w.heads_kv, ring_size=w.ring)
+        plan = self.plan
+        self.storage = make_qkv(w, seed=seed)
+        self.full = [self.to_dev(x) for x in self.storage]
+        self.shards = [plan.empty_seq_shards(), plan.empty_kv_seq_shards(), plan.empty_kv_seq_shards()]
+        self.out = plan.empty_seq_shards()
+        self.full_out = torch.empty(plan.full_shape(), dtype=plan.torch_dtype, device=dev)
+        self.ws = torch.empty(plan.workspace_bytes(n_chunks), dtype=torch.uint8, device=dev)
+        self.small = 3 * w.tensor_bytes <= 126 * 2**20
+        self.flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev) if self.small else None
+        self.ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(steps)]
+        self.graphs = []
+        self.launches_per_step = 0
+        self.use_graph = graph
+
+    def to_dev(self, x):
+        torch = self.torch
+        if self.w.dtype == "bf16":
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(self.dev)
+        return torch.from_numpy(x).to(self.dev)
+
+    def step(self, full=None, full_out=None):
+        usp, plan = self.usp, self.plan
+        for x, sh in zip(full or self.full, self.shards):
+            usp.scatter_sequence(plan, x, out=sh)
+        usp.ulysses_attention(plan, *self.shards, out=self.out, num_chunks=self.n_chunks, workspace=self.ws)
+        usp.gather_sequence(plan, self.out, out=self.full_out if full_out is None else full_out)
+
+    def prepare(self, warmup):
+        torch, usp = self.torch, self.usp
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            self.step()
+        for a, b in self.ev_a:
+            a.record(stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        if not self.use_graph:
+            return
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        before = usp.kernel_launches()
+        with torch.cuda.stream(cap):
+            for i in range(self.steps):
+                g = torch.cuda.CUDAGraph()
+                self.plan.set_timing_events(*self.ev_a[i])
+                with torch.cuda.graph(g, stream=cap):
+                    self.step()
+                self.graphs.append(g)
+            self.plan.set_timing_events(None, None)
+        self.launches_per_step = (usp.kernel_launches() - before) // self.steps
+        stream.wait_stream(cap)
+        for _ in range(2):
+            self.graphs[0].replay()
+        torch.cuda.synchronize()
+
+    def timed_pass(self, barrier=lambda: None):
+        """Times exactly `steps` steps between two synchronised barriers.
+        Returns (device ms of the steps, per-step attention ms, launches)."""
+        torch, usp = self.torch, self.usp
+        stream = torch.cuda.current_stream()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        launches0 = usp.kernel_launches()
+        t0.record(stream)
+        for i in range(self.steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            if self.graphs:
+                self.graphs[i].replay()
+            else:
+                self.plan.set_timing_events(*self.ev_a[i])
+                self.step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        self.plan.set_timing_events(None, None)
+        launches = usp.kernel_launches() - launches0 + self.launches_per_step * (self.steps if self.graphs else 0)
+        ms = t0.elapsed_time(t1) - self.flush_ms()
+        return ms, [a.elapsed_time(b) for a, b in self.ev_a], launches
+
+    def flush_ms(self):
+        if self.flush is None:
+            return 0.0
+        if not hasattr(self, "_flush_ms"):
+            torch = self.torch
+            stream = torch.cuda.current_stream()
+            fs, fe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for _ in range(3):
+                self.flush.zero_()
+            fs.record(stream)
+            for _ in range(self.steps):
+                self.flush.zero_()
+            fe.record(stream)
+            torch.cuda.synchronize()
+            self._flush_ms = fs.elapsed_time(fe)
+        return self._flush_ms
+
+    def attention_launches(self):
+        """Attention kernel launches per step (one per head chunk)."""
+        return len(self.usp.head_chunk_ranges(max(b - a for a, b in self.plan.head_ranges), self.n_chunks))
+
+    def close(self):
+        self.graphs.clear()
+        self.plan.close()
+        del self.full, self.shards, self.out, self.full_out, self.ws, self.flush
+        self.torch.cuda.empty_cache()
+
+
+def attention_roofline(w, attn_ms_step, n_launch, pk, pk_kind):
+    """The attention kernel against the bf16 tensor-core peak: FLOP of one
+    launch (4*B*H_launch*T'^2*D) over its average duration."""
+    flop = float(w.attention_flop)
+    achieved = flop / (attn_ms_step / 1e3) / 1e12  # the launches of a step run back to back
+    peak_key = "bf16_tflops_sustained"
+    return {"bound": "tensor", "achieved": achieved, "peak": pk[peak_key], "unit": "TFLOP/s",
+            "frac": achieved / pk[peak_key], "peak_source": f"{peak_key} ({pk_kind})",
+            "frac_of_burst_peak": achieved / pk["bf16_tflops"], "attention_ms_per_step": attn_ms_step,
+            "launch_ms": attn_ms_step / n_launch}
+
+
+# The other workloads of the benchmark, each measured on its own in the same
+# run (1 GPU): name -> (workload, head chunks).
+CONFIG_SWEEP = (
+    ("tiny_chunks1", W.TINY, 1),
+    ("tiny_chunks2", W.TINY, 2),
+    ("vit", W.VIT, 1),
+    ("chunked", W.CHUNKED, 3),
+    ("chunked_chunks1", W.CHUNKED, 1),
+    ("hybrid", W.HYBRID, 1),
+)
+
+
+def measure_config(usp, torch, dev, w, n_chunks, steps, warmup, pk, pk_kind, min_seconds=0.6, max_passes=200):
+    """One workload's step timed in passes of `steps` graph replays until
+    `min_seconds` of device time (so that the clock sampler sees the load);
+    reports the median pass. Block FLOP/s counts the whole step (scatter,
+    exchange, attention, gather); attention FLOP/s the attention kernels."""
+    bb = BlockBench(usp, torch, dev, w, n_chunks, steps, seed=w.seed)
+    try:
+        bb.prepare(warmup)
+        clocks = ClockSampler(dev.index or 0)
+        clocks.start()
+        passes, spent = [], 0.0
+        while (spent < min_seconds * 1e3 or len(passes) < 3) and len(passes) < max_passes:
+            ms, attn, launches = bb.timed_pass()
+            passes.append((ms, statistics.mean(attn), launches))
+            spent += ms
+        clk = clocks.stop()
+        assert usp.device_status() == 0, "a device-side wait ran out"
+        ms = statistics.median(p[0] for p in passes) / steps
+        attn = statistics.median(p[1] for p in passes)
+        flop = float(w.attention_flop)
+        entry = {"workload": w.name, "dtype": w.dtype, "num_chunks": n_chunks,
+                 "head_chunks": [list(c) for c in usp.head_chunk_ranges(
+                     max(b - a for a, b in bb.plan.head_ranges), n_chunks)],
+                 "ms_per_step": ms, "attention_ms_per_step": attn,
+                 "block_tflops": flop / (ms / 1e3) / 1e12, "attention_tflops": flop / (attn / 1e3) / 1e12,
+                 "gpu_launches_per_step": passes[0][2] // steps,
+                 "timing": f"median of {len(passes)} passes of {steps} CUDA-graph steps",
+                 "l2": "flushed (512 MiB write, subtracted) before every step" if bb.small
+                       else "inputs larger than L2", "clocks": clk}
+        if w.dtype != "fp32":
+            entry["block_frac_sustained"] = entry["block_tflops"] / pk["bf16_tflops_sustained"]
+            entry["block_frac_burst"] = entry["block_tflops"] / pk["bf16_tflops"]
+            entry["roofline"] = attention_roofline(w, attn, bb.attention_launches(), pk, pk_kind)
+        return entry
+    finally:
+        bb.close()
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -268,101 +458,18 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.set_device(dev)
     n_chunks = args.num_chunks or w.num_chunks[0]
     pk, pk_kind = peaks()
-    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix, kv_heads=w.heads_kv,
-                    ring_size=w.ring)
-    tdt = plan.torch_dtype
-    storage = make_qkv(w, seed=w.seed + 7919 * rank)
-
-    def to_dev(x):
-        if w.dtype == "bf16":
-            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(x).to(dev)
-
-    full = [to_dev(x) for x in storage]
-    shards = [plan.empty_seq_shards() for _ in range(3)]
-    out = plan.empty_seq_shards()
-    full_out = torch.empty(plan.full_shape(), dtype=tdt, device=dev)
-    ws = torch.empty(plan.workspace_bytes(n_chunks), dtype=torch.uint8, device=dev)
-    small = 3 * w.tensor_bytes <= 126 * 2**20
-    flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev) if small else None
-
-    def step():
-        for x, sh in zip(full, shards):
-            usp.scatter_sequence(plan, x, out=sh)
-        usp.ulysses_attention(plan, *shards, out=out, num_chunks=n_chunks, workspace=ws)
-        usp.gather_sequence(plan, out, out=full_out)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    # The step's calls are stream-ordered and synchronise nothing, so the whole
-    # step can be captured and replayed as a CUDA graph (this removes the host
-    # launch cost, which dominates the small workloads). One graph is captured
-    # per timed step, each with its own pair of attention timing events.
-    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in ev_a:
-        a.record(stream)
-        b.record(stream)
-    torch.cuda.synchronize()
-    graphs = []
-    launches_per_step = 0
-    if not args.no_graph:
-        cap = torch.cuda.Stream()
-        cap.wait_stream(stream)
-        before = usp.kernel_launches()
-        with torch.cuda.stream(cap):
-            for i in range(args.steps):
-                g = torch.cuda.CUDAGraph()
-                plan.set_timing_events(*ev_a[i])
-                with torch.cuda.graph(g, stream=cap):
-                    step()
-                graphs.append(g)
-            plan.set_timing_events(None, None)
-        launches_per_step = (usp.kernel_launches() - before) // args.steps
-        stream.wait_stream(cap)
-        for _ in range(2):
-            graphs[0].replay()
-        torch.cuda.synchronize()
-
-    # timed region: K steps, attention kernels bracketed by their own events
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bb = BlockBench(usp, torch, dev, w, n_chunks, args.steps, seed=w.seed + 7919 * rank, graph=not args.no_graph)
+    bb.prepare(args.warmup)
+    # timed region: exactly K steps, attention kernels bracketed by their own events
     clocks = ClockSampler(local_rank)
     clocks.start()
-    torch.cuda.synchronize()
-    barrier()
-    launches0 = usp.kernel_launches()
-    flush_ms = 0.0
-    t0.record(stream)
-    for i in range(args.steps):
-        if flush is not None:
-            flush.zero_()
-        if graphs:
-            graphs[i].replay()
-        else:
-            plan.set_timing_events(*ev_a[i])
-            step()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    launches = usp.kernel_launches() - launches0 + launches_per_step * (args.steps if graphs else 0)
-    barrier()
+    ms_total, attn_ms, launches = bb.timed_pass(barrier)
     clk = clocks.stop()
-    plan.set_timing_events(None, None)
-    ms_total = t0.elapsed_time(t1)
-    if flush is not None:
-        fs, fe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        fs.record(stream)
-        for _ in range(args.steps):
-            flush.zero_()
-        fe.record(stream)
-        torch.cuda.synchronize()
-        flush_ms = fs.elapsed_time(fe)
-        ms_total -= flush_ms
-    attn_ms = [a.elapsed_time(b) for a, b in ev_a]
     assert usp.device_status() == 0, "a device-side wait ran out"
 
     ms_max, attn_ms_max = reduce_max([ms_total, statistics.mean(attn_ms)], world, dev)
@@ -372,23 +479,20 @@ def run_ours(args, w, rank, world, local_rank):
 
     line = None
     if rank == 0:
-        n_launch_attn = len(usp.head_chunk_ranges(max(b - a for a, b in plan.head_ranges), n_chunks))
-        attn_launch_ms = attn_ms_max / n_launch_attn
-        achieved = flop / n_launch_attn / (attn_launch_ms / 1e3) / 1e12
-        peak_key = "bf16_tflops_sustained"
+        n_launch_attn = bb.attention_launches()
+        roof = attention_roofline(w, attn_ms_max, n_launch_attn, pk, pk_kind)
         # algorithmic bytes of one launch: q, k, v read once and o written once
-        traffic = recorded_traffic("attention", 4 * w.tensor_bytes / n_launch_attn)
+        roof["traffic"] = recorded_traffic("attention", 4 * w.tensor_bytes / n_launch_attn)
+        roof["kernel"] = "attn_tc_kernel (tcgen05), one launch per head chunk"
+        roof["peak_source"] += "; the kernel runs inside a long step loop"
+        roof = {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "kernel",
+                                     "peak_source", "frac_of_burst_peak", "attention_ms_per_step", "launch_ms")}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {**workload_config(w, n_chunks, world), "cuda_graph": bool(graphs)},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk[peak_key], "unit": "TFLOP/s",
-                         "frac": achieved / pk[peak_key], "traffic": traffic,
-                         "kernel": "attn_tc_kernel (tcgen05), one launch per head chunk",
-                         "peak_source": f"{peak_key} ({pk_kind}); the kernel runs inside a long step loop",
-                         "frac_of_burst_peak": achieved / pk["bf16_tflops"],
-                         "attention_ms_per_step": attn_ms_max},
+            "config": {**workload_config(w, n_chunks, world), "cuda_graph": bool(bb.graphs)},
+            "roofline": roof,
             "gpu_launches": int(launches),
             "clocks": clk,
         }
@@ -399,18 +503,14 @@ def run_ours(args, w, rank, world, local_rank):
     # way a caller streaming batches from host memory would run them; the
     # timed region spans the first input copy to the last output copy.
     if not args.no_e2e:
-        host_in = [torch.from_numpy(x.view(np.int16) if w.dtype == "bf16" else x).pin_memory() for x in storage]
-        host_out = torch.empty(full_out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
+        stream = torch.cuda.current_stream()
+        host_in = [torch.from_numpy(x.view(np.int16) if w.dtype == "bf16" else x).pin_memory() for x in bb.storage]
+        host_out = torch.empty(bb.full_out.shape,
+                               dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
         k_e2e = max(2, args.steps)
-        fins = [full, [torch.empty_like(x) for x in full]]
-        fouts = [full_out, torch.empty_like(full_out)]
+        fins = [bb.full, [torch.empty_like(x) for x in bb.full]]
+        fouts = [bb.full_out, torch.empty_like(bb.full_out)]
         s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
-
-        def step_on(fi, fo):
-            for x, sh in zip(fi, shards):
-                usp.scatter_sequence(plan, x, out=sh)
-            usp.ulysses_attention(plan, *shards, out=out, num_chunks=n_chunks, workspace=ws)
-            usp.gather_sequence(plan, out, out=fo)
 
         def e2e_run(nsteps):
             ev = lambda: torch.cuda.Event()  # noqa: E731
@@ -430,7 +530,7 @@ def run_ours(args, w, rank, world, local_rank):
                 stream.wait_event(h2d_done[i])
                 if i >= 2:
                     stream.wait_event(d2h_done[i - 2])  # output buffer b has been copied out
-                step_on(fins[b], fouts[b])
+                bb.step(fins[b], fouts[b])
                 comp_done[i].record(stream)
                 with torch.cuda.stream(s_d2h):
                     s_d2h.wait_event(comp_done[i])
@@ -455,11 +555,32 @@ def run_ours(args, w, rank, world, local_rank):
                            "pipeline": "double-buffered: H2D of step i+1 and D2H of step i-1 overlap step i "
                                        "on separate streams; timed from the first H2D to the last D2H"}
         del host_in, host_out, fins, fouts
-    del graphs
-    plan.close()
-    del full, shards, out, full_out, ws
-    torch.cuda.empty_cache()
+    storage = bb.storage
+    headline_entry = None
+    if rank == 0:
+        headline_entry = {"workload": w.name, "dtype": w.dtype, "num_chunks": n_chunks,
+                          "ms_per_step": ms_step, "attention_ms_per_step": attn_ms_max,
+                          "block_tflops": value / world, "attention_tflops": line["roofline"]["achieved"],
+                          "block_frac_sustained": value / world / pk["bf16_tflops_sustained"],
+                          "block_frac_burst": value / world / pk["bf16_tflops"],
+                          "roofline": {k: line["roofline"][k] for k in ("achieved", "frac", "frac_of_burst_peak")},
+                          "timing": "the headline's own timed region (this line's value)", "clocks": clk}
+    bb.close()
 
+    if rank == 0 and world == 1 and not args.no_configs:
+        configs = {w.name.split("-")[0]: headline_entry}
+        for name, cw, cn in CONFIG_SWEEP:
+            if cw.name == w.name and cn == n_chunks:
+                continue
+            configs[name] = measure_config(usp, torch, dev, cw, cn, args.steps, args.warmup, pk, pk_kind)
+        c3, c1 = configs.get("chunked"), configs.get("chunked_chunks1")
+        if c3 and c1:
+            configs["chunk_overlap"] = {
+                "what": "the head-chunked workload's block with num_chunks=3 (chunk c+1's exchange on the "
+                        "plan's second stream under chunk c's attention) against num_chunks=1, same run",
+                "speedup_block": c1["ms_per_step"] / c3["ms_per_step"],
+                "ms_per_step_chunks3": c3["ms_per_step"], "ms_per_step_chunks1": c1["ms_per_step"]}
+        line["configs"] = configs
     if rank == 0 and world == 1 and not args.no_reshard:
         line["reshard"] = reshard_measurement(usp, torch, dev, pk, pk_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -130,3 +130,12 @@ def test_header_compiles_and_links_from_c(usp, tmp_path):
                    check=True)
     usage = subprocess.run([str(out)], capture_output=True, text=True)
     assert usage.returncode == 2 and "usage" in usage.stderr
+
+
+def test_noalloc_scratch_size_matches_header(usp):
+    """The binding's copy of the allocation-free scratch size is the header's."""
+    import re
+    with open(os.path.join(ROOT, "include", "usp.h")) as f:
+        m = re.search(r"#define USP_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", f.read())
+    assert m, "USP_NOALLOC_SCRATCH_BYTES not found in include/usp.h"
+    assert usp.NOALLOC_SCRATCH_BYTES == int(m[1]) * int(m[2]) * int(m[3])

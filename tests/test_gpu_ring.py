@@ -13,8 +13,9 @@ import torch
 from oracle import layout as ol
 from oracle import ring as oring
 from tests.gpu_util import assert_close, to_device, to_f64
-from ulysses_sequence_attention_sp_b200.synth import make_qkv, storage_to_f64
-from ulysses_sequence_attention_sp_b200.workloads import Workload
+from oracle.attention import default_scale
+from ulysses_sequence_attention_sp_b200.synth import bf16_bits_to_f32, make_qkv, storage_to_f64
+from ulysses_sequence_attention_sp_b200.workloads import HYBRID, Workload
 
 pytestmark = pytest.mark.gpu
 
@@ -197,3 +198,91 @@ def test_hybrid_replays_from_a_cuda_graph(usp, mode):
     assert usp.device_status() == 0
     del graph
     plan.close()
+
+
+def _hybrid_sample_rows(plan, groups, rng, n_random=24):
+    """Every rank boundary, both edges of every ring block, first and last
+    rows, and seeded random rows (full-sequence row numbers)."""
+    rows = {0, 1, plan.tokens - 1, plan.tokens - 2}
+    for t0, t1 in plan.token_ranges:
+        rows.update(plan.prefix + t for t in (t0 - 1, t0, t1 - 1) if 0 <= t < plan.seq_len)
+    for _members, (b0, b1), _local in groups:
+        rows.update(plan.prefix + t for t in (b0 - 1, b0, b0 + 1, b1 - 2, b1 - 1, b1) if 0 <= t < plan.seq_len)
+    rows.update(int(x) for x in rng.integers(0, plan.tokens, size=n_random))
+    return sorted(rows)
+
+
+def test_full_size_hybrid_sampled_rows(usp):
+    """The video latent as Ulysses 4 x Ring 2 (T=75600, H=24, D=128, two ring
+    blocks of 37,800 keys, each ending in a ragged 256-key tile), in the
+    launch configuration the benchmark times. Sampled rows of every head are
+    computed by the oracle's ring steps: the row's own block first, then the
+    previous ring block, each normalised over its keys with its log-sum-exp,
+    merged by log-sum-exp weights."""
+    w = HYBRID
+    ring, uly = w.ring, w.world // w.ring
+    storage, plan, out = _run(usp, w, ring, w.num_chunks[0])
+    for o in out:
+        assert not torch.isnan(o).any().item(), "an output element was never written"
+    q, k, v = storage
+    groups = oring.ring_groups(plan.token_ranges, uly, ring)
+    rows = _hybrid_sample_rows(plan, groups, np.random.default_rng(8))
+    assert 37799 in rows and 37800 in rows
+
+    def block_rows(gp):
+        b0, b1 = groups[gp][1]
+        keys = np.arange(plan.prefix + b0, plan.prefix + b1)
+        return np.concatenate([np.arange(plan.prefix), keys]) if gp == 0 else keys
+
+    def group_of(t):
+        tok = t - plan.prefix
+        return 0 if tok < 0 else next(g for g, (_m, (b0, b1), _l) in enumerate(groups) if b0 <= tok < b1)
+
+    scale = default_scale(w.head_dim)
+    got_all, ref_all = [], []
+    for b in range(w.batch):
+        for h in range(w.heads):
+            kh = storage_to_f64(k[b, :, h], w.dtype)
+            vh = storage_to_f64(v[b, :, h], w.dtype)
+            for g in range(ring):
+                rows_g = [t for t in rows if group_of(t) == g]
+                qh = storage_to_f64(q[b, rows_g, h], w.dtype)
+                o = lse = None
+                for step in range(ring):
+                    keys = block_rows((g - step) % ring)
+                    o_s, lse_s = oring.block_attention(qh, kh[keys], vh[keys], scale)
+                    o, lse = (o_s, lse_s) if o is None else oring.merge_partials(o, lse, o_s, lse_s)
+                for i, t in enumerate(rows_g):
+                    tok = t - plan.prefix
+                    owners = range(w.world) if tok < 0 else [
+                        next(r for r, (a, c) in enumerate(plan.token_ranges) if a <= tok < c)]
+                    for r in owners:
+                        local = t if tok < 0 else plan.prefix + tok - plan.token_ranges[r][0]
+                        got_all.append(to_f64(out[r][b, local, h], w.dtype))
+                        ref_all.append(o[i])
+    st = assert_close(np.stack(got_all), np.stack(ref_all), w.dtype, w.name)
+    print(w.name, len(rows), "rows x", w.heads, "heads", st)
+    plan.close()
+
+
+def test_full_size_hybrid_every_element_against_fp32_kernel(usp):
+    """Secondary signal at full size: every output element of the hybrid block
+    against the fp32 CUDA-core kernel's ring walk on the same values (the bf16
+    inputs upcast exactly), with the bf16 tolerances."""
+    w = HYBRID
+    storage, plan, out = _run(usp, w, w.ring, w.num_chunks[0])
+    plan32 = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, "fp32", w.prefix, ring_size=w.ring)
+    shards32 = [usp.scatter_sequence(plan32, torch.from_numpy(bf16_bits_to_f32(x)).cuda()) for x in storage]
+    del storage
+    out32 = usp.ulysses_attention(plan32, *shards32)
+    torch.cuda.synchronize()
+    assert usp.device_status() == 0
+    for r in range(w.world):
+        got, ref = out[r].double(), out32[r].double()
+        diff = (got - ref).abs()
+        st = {"max_abs": diff.max().item(), "mean_abs": diff.mean().item(),
+              "rel_l2": ((got - ref).norm() / ref.norm()).item(), "nan": int(torch.isnan(got).sum().item())}
+        assert st["nan"] == 0 and st["max_abs"] <= 2e-2 and st["mean_abs"] <= 2e-3 and st["rel_l2"] <= 1e-2, (r, st)
+    print(w.name, "rank", w.world - 1, st)
+    plan.close()
+    plan32.close()

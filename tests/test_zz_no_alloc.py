@@ -27,6 +27,11 @@ pytestmark = pytest.mark.gpu
 CASES = [
     Workload("noalloc-bf16-T1000-cls-H6-D128-P4", 1, 1000, 1, 6, 128, 4, "bf16", 1.0, 9101, (1, 2)),
     Workload("noalloc-bf16-B3-T300-H5-D80-P3", 3, 300, 0, 5, 80, 3, "bf16", 0.5, 9102, (1, 3)),
+    # grouped-query attention: 8 query heads over 4 kv heads (separate kv head ranges in the scratch)
+    Workload("noalloc-gqa-bf16-T700-H8-KV4-D64-P4", 1, 700, 0, 8, 64, 4, "bf16", 1.0, 9103, (1, 2), kv_heads=4),
+    # Ulysses 2 x Ring 2 hybrid with a cls row (ring key blocks in the scratch)
+    Workload("noalloc-hybrid-bf16-T900-cls-H4-D128-U2xR2", 1, 900, 1, 4, 128, 4, "bf16", 1.0, 9104, (1, 2),
+             ring=2),
 ]
 
 
@@ -50,14 +55,22 @@ def _noalloc_call(usp, plan, q, k, v, out, num_chunks):
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_noalloc_matches_regular_entry_point_twice(usp, w):
-    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix)
+    plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix, kv_heads=w.heads_kv,
+                    ring_size=w.ring)
     for call, seed in enumerate((w.seed, w.seed + 1)):
         num_chunks = w.num_chunks[call % len(w.num_chunks)]
         shards = [usp.scatter_sequence(plan, to_device(x, w.dtype)) for x in make_qkv(w, seed)]
         ref = usp.ulysses_attention(plan, *shards, num_chunks=num_chunks)
         got = plan.empty_seq_shards(fill=float("nan"))
+        torch.cuda.synchronize()
+        # the call itself reserves no device memory: neither torch's allocator
+        # nor the device's free memory moves across it
+        allocated, free = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         assert _noalloc_call(usp, plan, *shards, got, num_chunks) == usp.USP_OK, usp._lib.usp_last_error_message()
         torch.cuda.synchronize()
+        if call == 1:  # the first call may still load kernels' code on first use
+            assert torch.cuda.memory_allocated() == allocated
+            assert torch.cuda.mem_get_info()[0] == free
         assert usp.device_status() == 0
         for r in range(plan.world):
             assert_close(to_f64(got[r], w.dtype), to_f64(ref[r], w.dtype), w.dtype, f"call {call} rank {r}")
