@@ -15,6 +15,16 @@
  *  - Every launch goes on the caller's stream (`stream`, a cudaStream_t; NULL
  *    is the legacy default stream). No call synchronises the host, except
  *    usp_device_status(). Calls are stream-ordered like any CUDA kernel.
+ *  - Threads and streams: one plan may serve calls from several host threads
+ *    and on several streams at once. Each call enqueues its work (including
+ *    the event records and waits of usp_ulysses_attention's chunk overlap on
+ *    the plan's auxiliary stream) under the plan's lock, so calls never
+ *    cross-wire each other's dependencies; work of different calls is then
+ *    ordered only by the streams it runs on. Calls that may run at the same
+ *    time on the GPU must not share an output or a workspace buffer (the
+ *    allocation-free entry point shares one scratch array: see there).
+ *    Plan set-up calls (usp_plan_set_*) must not race with calls using the
+ *    plan.
  *  - Tensors are dense and contiguous, row-major, in the BSHD layout of the
  *    ragged transport page: [batch, tokens, heads, head_dim]. Pointers must be
  *    16-byte aligned (USP_ERR_ALIGN otherwise); there is no slow path.
@@ -102,7 +112,10 @@ int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_ou
  * `dtype`, with `prefix_tokens` (0 or 1) replicated leading tokens
  * ("deepspeed/sequence/autosp_vit.py": the cls token is replicated on every
  * rank). Binds the plan to the current CUDA device and creates one auxiliary
- * stream and its events there (used to overlap head chunks).
+ * stream and its events there (used to overlap head chunks), and looks up the
+ * device address of usp_ulysses_attention_noalloc's scratch array there
+ * (loading the library module that holds it reserves that array on the device,
+ * once per process and device).
  * Errors: USP_ERR_INVALID_ARG (world < 1 or > USP_MAX_WORLD, seq_len < world,
  * heads < world or > USP_MAX_HEADS, batch < 1, head_dim < 1, prefix not 0/1),
  * USP_ERR_DTYPE, USP_ERR_NO_DEVICE, USP_ERR_CUDA.
@@ -351,17 +364,130 @@ int usp_ulysses_attention_lse(const usp_plan* plan, const void* const* q, const 
  * cudaMalloc or cudaFree call and uses no allocating library routine.
  *  - Plans whose usp_ulysses_attention_workspace_size exceeds the array are
  *    rejected with USP_ERR_SHAPE before any launch.
- *  - The first call on a device looks up the array's device address there
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture.
+ *  - The array's device address is looked up (cudaGetSymbolAddress) when the
+ *    plan is created, with the plan's device current, and kept in the plan; so
+ *    the array is reserved on a device no later than the first plan created
+ *    there, and this call itself loads nothing. A plan does not outlive the
+ *    CUDA context it was created in (after a device reset, create new plans).
  *  - All calls share the one array and it keeps the last call's contents.
- *    Calls that overlap on the GPU (other streams, other host threads) race on
- *    it: order them. Nothing in it has to start at zero.
+ *    Calls that overlap on the GPU (other streams, other host threads, other
+ *    plans on the same device) race on it: order them. Nothing in it has to
+ *    start at zero.
  */
 #define USP_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int usp_ulysses_attention_noalloc(const usp_plan* plan, const void* const* q, const void* const* k,
                                   const void* const* v, void* const* out, float scale, int32_t num_chunks,
                                   void* stream);
+
+/*
+ * Rank-local entry points: the Ulysses block across processes, one process
+ * (one GPU) per sequence-parallel rank. "h3_blackwell_runtime/distributed.py
+ * -- Ragged Ulysses sequence-parallel transport", seq_to_heads / heads_to_seq:
+ * each rank packs one contiguous block per peer, the blocks travel in one
+ * ragged all-to-all (all_to_all_single with per-peer element counts), and each
+ * rank unpacks what it receives in source-rank order. API page,
+ * ulysses_attention(prefer_all_gather): the same result through equal-size
+ * all-gathers (blocks padded to the longest), which a captured CUDA graph can
+ * replay. The library packs, unpacks and computes; the caller runs the
+ * collective (e.g. NCCL through torch.distributed) on buffers it owns.
+ *
+ * Every rank creates the same plan (same sizes, world = number of ranks) on
+ * its own device and passes its rank; only plain and grouped-query plans are
+ * taken (a Ulysses + Ring plan returns USP_ERR_UNSUPPORTED). Head chunks are
+ * usp_head_chunk_ranges(G = H_0, num_chunks); chunk c exchanges, on every
+ * rank j, the query heads of j inside the chunk's local window (n_j of them)
+ * and the kv heads whose first query head lies there (m_j; m_j = n_j without
+ * grouped-query attention).
+ *
+ * Wire format, in elements of the plan's type (p = prefix rows, T_i = rank i's
+ * tokens, T' = p + T; every block is row-major [B][rows][heads][D]):
+ *   USP_DIST_SEQ_TO_HEAD  rank r -> peer j: q [B][p+T_r][n_j][D], then, with
+ *       ntensors = 3, k and v [B][p+T_r][m_j][D]. Every rank sends its prefix
+ *       rows; receivers keep rank 0's.
+ *   USP_DIST_HEAD_TO_SEQ  rank r -> peer j: o [B][p+T_j][n_r][D] (the prefix
+ *       rows go to every peer).
+ *   USP_DIST_GATHER_SEQ   rank r's all-gather block: its q, k, v sequence
+ *       shards back to back ([B][p+T_r][H][D], then [B][p+T_r][Hkv][D] twice),
+ *       padded to the longest block over ranks (chunk-independent).
+ *   USP_DIST_GATHER_HEADS rank r's all-gather block: o [B][T'][n_r][D],
+ *       padded to the longest block over ranks.
+ * A block's padding is never read.
+ */
+#define USP_DIST_SEQ_TO_HEAD 0
+#define USP_DIST_HEAD_TO_SEQ 1
+#define USP_DIST_GATHER_SEQ 2
+#define USP_DIST_GATHER_HEADS 3
+
+/*
+ * usp_dist_exchange_counts -- the split lists of one exchange for `rank`
+ * (transport page, seq_to_heads: input_splits / output_splits), in elements,
+ * computed from the sizes alone (no device is needed, so a host-side
+ * collective can be planned anywhere). world arrays: send_counts[j] and
+ * send_displs[j] for peer j, recv_counts[i] and recv_displs[i] for source i.
+ * All-to-all kinds: displacements are the running sums of the counts. Gather
+ * kinds: every count is the padded block, send_displs are 0 and
+ * recv_displs[i] = i * block (all_gather_into_tensor's layout).
+ * Errors: as usp_plan_create_gqa for the sizes; USP_ERR_INVALID_ARG for a rank
+ * outside [0, world), an unknown exchange, ntensors other than 1 or 3
+ * (q/k/v kinds) or 1 (output kinds), num_chunks < 1 or a chunk outside the
+ * head chunks; NULL outputs.
+ */
+int usp_dist_exchange_counts(int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv, int32_t head_dim,
+                             int32_t world, int32_t prefix_tokens, int32_t rank, int32_t exchange, int32_t ntensors,
+                             int32_t num_chunks, int32_t chunk, int64_t* send_counts, int64_t* send_displs,
+                             int64_t* recv_counts, int64_t* recv_displs);
+
+/*
+ * usp_dist_pack -- fills `send` (usp_dist_exchange_counts' send layout) for
+ * chunk `chunk` of `num_chunks`:
+ *   SEQ_TO_HEAD   in[t] = this rank's sequence shard of q, k, v
+ *                 ([B][p+T_r][H or Hkv][D]); ntensors 1 (q) or 3.
+ *   HEAD_TO_SEQ   in[0] = this rank's head shard o [B][T'][H_r][D].
+ *   GATHER_SEQ    in[t] as SEQ_TO_HEAD (copied whole; the chunk is ignored).
+ *   GATHER_HEADS  in[0] as HEAD_TO_SEQ.
+ * Device pointers, 16-byte aligned, caller-owned; send must not overlap in.
+ * Errors: as usp_dist_exchange_counts, plus USP_ERR_ALIGN and USP_ERR_CUDA.
+ */
+int usp_dist_pack(const usp_plan* plan, int32_t rank, int32_t exchange, int32_t ntensors, int32_t num_chunks,
+                  int32_t chunk, const void* const* in, void* send, void* stream);
+
+/*
+ * usp_dist_unpack -- reads `recv` (usp_dist_exchange_counts' receive layout,
+ * after the collective) for chunk `chunk` of `num_chunks`:
+ *   SEQ_TO_HEAD, GATHER_SEQ  out[t] = this rank's head shards of q, k, v
+ *                 [B][T'][H_r or Hkv_r][D]; the chunk's heads are written (all
+ *                 chunks in order fill the shards).
+ *   HEAD_TO_SEQ, GATHER_HEADS  out[0] = this rank's sequence shard
+ *                 [B][p+T_r][H][D]; the chunk's heads of every rank are written.
+ * Errors as usp_dist_pack.
+ */
+int usp_dist_unpack(const usp_plan* plan, int32_t rank, int32_t exchange, int32_t ntensors, int32_t num_chunks,
+                    int32_t chunk, const void* recv, void* const* out, void* stream);
+
+/*
+ * usp_dist_workspace_size -- bytes of workspace usp_dist_attention needs on
+ * `rank`: (H_r + 2 Hkv_r) * B * T' * D elements, each part 256-byte aligned.
+ */
+int usp_dist_workspace_size(const usp_plan* plan, int32_t rank, size_t* bytes);
+
+/*
+ * usp_dist_attention -- API page, ulysses_attention's run_attention on one
+ * rank, for the heads of chunk `chunk`: `recv` holds the received q, k, v
+ * (exchange USP_DIST_SEQ_TO_HEAD with ntensors 3, or USP_DIST_GATHER_SEQ);
+ * they are unpacked into `workspace` and attended (non-causal softmax
+ * attention over all T' tokens, as usp_head_attention), and the epilogue
+ * writes the output straight into `send_o` in the layout of the way back:
+ * USP_DIST_HEAD_TO_SEQ blocks (row t to the block of the peer owning token t)
+ * for SEQ_TO_HEAD, or this rank's USP_DIST_GATHER_HEADS block for GATHER_SEQ.
+ * scale <= 0 selects 1/sqrt(D). workspace: at least usp_dist_workspace_size()
+ * bytes, 256-byte aligned; its contents are scratch, but with grouped-query
+ * attention a kv head shared by two chunks arrives with the first of them, so
+ * a block's chunks must run in order on the same workspace. Errors as
+ * usp_dist_pack, plus those of usp_ulysses_attention's attention.
+ */
+int usp_dist_attention(const usp_plan* plan, int32_t rank, int32_t exchange, int32_t num_chunks, int32_t chunk,
+                       const void* recv, void* send_o, float scale, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /*
  * usp_ulysses_attention_graph_create -- captures one usp_ulysses_attention

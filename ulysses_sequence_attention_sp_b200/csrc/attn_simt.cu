@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
   const float inv_l = 1.f / l;
   for (int s = seg_lo; s < seg_hi; ++s) {
     const int64_t rows_s = out.prefix + out.seg_len[s];
-    const int64_t base = ((b * rows_s + row_in_seg) * out.out_heads + hm) * D;
+    const int64_t base = ((b * rows_s + row_in_seg) * out.out_heads + hm - out.head_base) * D;
     float* dst = static_cast<float*>(out.seg_ptr[s]) + base;
     const int64_t ext = static_cast<int64_t>(L.batch) * rows_s * out.out_heads * D;  // bounds-checking builds
 #pragma unroll
@@ -145,11 +145,10 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(const __grid_consta
 template <int DPT>
 int launch_dpt(const AttnLaunch& L, cudaStream_t stream) {
   const size_t smem = 2 * kKT * DPT * kTPR * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<DPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(simt smem)");
-  }
+  if (smem > 48 * 1024)
+    if (int rc = ensure_smem_limit(reinterpret_cast<const void*>(attn_simt_kernel<DPT>), smem,
+                                   "cudaFuncSetAttribute(simt smem)"))
+      return rc;
   const float scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
   SimtBlocks B;
   const int kv_tokens = L.kv_tokens > 0 ? L.kv_tokens : L.tokens;

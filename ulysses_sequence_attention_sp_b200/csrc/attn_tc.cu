@@ -200,13 +200,6 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, int item) {
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return bf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
-// Exact float values of a packed bf16x2 / f16x2 word (lo = bits 0-15).
-__device__ __forceinline__ float2 unpack2(uint32_t w, bool bf16) {
-  if (bf16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-  __half2 h = *reinterpret_cast<__half2*>(&w);
-  return __half22float2(h);
-}
-
 template <int D, bool BF16, bool RING>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   using C = Cfg<D>;
@@ -609,7 +602,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         w1.w = pack2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l, BF16);
         for (int sg = seg_lo; sg < seg_hi; ++sg) {
           const int64_t rows_s = out.prefix + out.seg_len[sg];
-          const int64_t elem = ((static_cast<int64_t>(b) * rows_s + row_in_seg) * out.out_heads + hm) * D + c * 16;
+          const int64_t elem =
+              ((static_cast<int64_t>(b) * rows_s + row_in_seg) * out.out_heads + hm - out.head_base) * D + c * 16;
           if (!in_bounds(elem, 16, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 21, &g_attn_bounds))
             continue;
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem);
@@ -986,7 +980,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_persistent_kernel(const _
           for (int sg = lo; sg < hi; ++sg) {
             const int64_t rows_s = out.prefix + out.seg_len[sg];
             const int64_t elem =
-                ((static_cast<int64_t>(b) * rows_s + r_in) * out.out_heads + hm) * D + c * 16 + (lane & 1) * 8;
+                ((static_cast<int64_t>(b) * rows_s + r_in) * out.out_heads + hm - out.head_base) * D + c * 16 +
+                (lane & 1) * 8;
             if (!in_bounds(elem, 8, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 21, &g_attn_bounds))
               continue;
             *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem) = val;
@@ -1162,15 +1157,11 @@ template <int D, bool BF16>
 int launch_d(const AttnLaunch& L, cudaStream_t stream) {
   using C = Cfg<D>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory above the 227 KB per-CTA limit");
-  static bool configured = false;
-  if (!configured) {
-    for (auto* fn : {attn_tc_kernel<D, BF16, false>, attn_tc_kernel<D, BF16, true>,
-                     attn_tc_persistent_kernel<D, BF16, false>, attn_tc_persistent_kernel<D, BF16, true>}) {
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-      if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(attention smem)");
-    }
-    configured = true;
-  }
+  for (auto* fn : {attn_tc_kernel<D, BF16, false>, attn_tc_kernel<D, BF16, true>,
+                   attn_tc_persistent_kernel<D, BF16, false>, attn_tc_persistent_kernel<D, BF16, true>})
+    if (int rc = ensure_smem_limit(reinterpret_cast<const void*>(fn), C::SMEM_BYTES,
+                                   "cudaFuncSetAttribute(attention smem)"))
+      return rc;
   TcParams p;
   memset(&p, 0, sizeof(p));
   int rc;

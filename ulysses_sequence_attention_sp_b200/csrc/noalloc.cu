@@ -15,8 +15,6 @@
 // the last call's contents; nothing in it needs to start at zero, because
 // every call writes each element it later reads (the seq->head exchange
 // fills the q, k and v head shards before the attention reads them).
-#include <mutex>
-
 #include "usp_internal.h"
 
 namespace {
@@ -25,27 +23,20 @@ constexpr size_t kScratchBytes = static_cast<size_t>(USP_NOALLOC_SCRATCH_BYTES);
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device. In host
-// code the array's name is only a host-side stand-in, never a device address.
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
 
-int scratch_address(int device, void** out) {
-  if (device < 0 || device >= kMaxDevices)
-    return usp::set_error(USP_ERR_UNSUPPORTED, "device ordinal %d is beyond %d", device, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[device]) {
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return usp::cuda_check(e, "cudaGetSymbolAddress(scratch)");
-    g_scratch_ptr[device] = ptr;
-  }
-  *out = g_scratch_ptr[device];
+// In host code the array's name is only a host-side stand-in, never a device
+// address: the address is looked up on the current device, once per plan, when
+// the plan is created (usp_plan_create*), and kept in the plan, which lives no
+// longer than the CUDA context it was made in. The lookup loads this file's
+// module if it is not loaded yet, which is when the array is reserved.
+int usp::noalloc_scratch_lookup(void** out) {
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess) return usp::cuda_check(e, "cudaGetSymbolAddress(allocation-free scratch)");
+  *out = ptr;
   return USP_OK;
 }
-
-}  // namespace
 
 extern "C" int usp_ulysses_attention_noalloc(const usp_plan* plan, const void* const* q, const void* const* k,
                                              const void* const* v, void* const* out, float scale,
@@ -58,10 +49,7 @@ extern "C" int usp_ulysses_attention_noalloc(const usp_plan* plan, const void* c
                           "usp_ulysses_attention_noalloc: this plan needs %zu bytes of scratch, above the fixed "
                           "%zu-byte array; use usp_ulysses_attention with a caller-owned workspace",
                           need, kScratchBytes);
-  int device = 0;
-  cudaError_t e = cudaGetDevice(&device);
-  if (e != cudaSuccess) return usp::cuda_check(e, "cudaGetDevice");
-  void* scratch = nullptr;
-  if (int rc = scratch_address(device, &scratch)) return rc;
-  return usp_ulysses_attention(plan, q, k, v, out, scale, num_chunks, scratch, kScratchBytes, stream);
+  if (!plan->noalloc_scratch) return usp::set_error(USP_ERR_INVALID_ARG, "plan has no scratch address");
+  return usp_ulysses_attention(plan, q, k, v, out, scale, num_chunks, plan->noalloc_scratch, kScratchBytes,
+                               stream);
 }

@@ -203,10 +203,15 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
   p.nsel = a.nsel;
   p.outer = static_cast<int32_t>(a.outer);
   int32_t min_cnt = INT32_MAX;
+  if (a.prefix > 0 && a.tok_start[0] != 0)
+    return set_error(USP_ERR_INVALID_ARG, "internal: TMA pack with prefix rows needs source 0's tokens to start at 0");
   for (int s = 0; s < a.n_seq; ++s) {
-    p.r0[s] = s == 0 ? 0 : a.prefix;
-    p.cnt[s] = static_cast<int32_t>(s == 0 ? a.prefix + a.tok_len[s] : a.tok_len[s]);
-    p.d0[s] = static_cast<int32_t>(s == 0 ? 0 : a.prefix + a.tok_start[s]);
+    // Source 0's prefix rows and token rows form one run from head-side row 0
+    // (its tokens start at token 0); other sources skip their prefix rows.
+    const bool whole = s == 0 && a.prefix > 0;
+    p.r0[s] = whole ? 0 : a.prefix;
+    p.cnt[s] = static_cast<int32_t>(whole ? a.prefix + a.tok_len[s] : a.tok_len[s]);
+    p.d0[s] = static_cast<int32_t>(whole ? 0 : a.prefix + a.tok_start[s]);
     if (p.cnt[s] < min_cnt) min_cnt = p.cnt[s];
   }
   // Head units per tile: the largest common divisor of the buffers' selected
@@ -244,14 +249,14 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
   p.chunk_prefix[0] = 0;
   for (int s = 0; s < a.n_seq; ++s) p.chunk_prefix[s + 1] = p.chunk_prefix[s] + (p.cnt[s] + p.rows - 1) / p.rows;
   for (int i = 0; i < a.nsel; ++i) {
-    p.sel_head[i] = a.sel_head[i];
+    p.sel_head[i] = static_cast<uint16_t>(a.sel_head[i] - a.seq_unit_base);
     p.sel_rank[i] = a.sel_rank[i];
     p.sel_local[i] = static_cast<uint16_t>(a.sel_head[i] - a.head_start[a.sel_rank[i]]);
   }
   p.total_units = static_cast<int64_t>(a.ntensors) * a.outer * p.chunk_prefix[a.n_seq] * p.ngroups;
   p.heads = a.heads;
   p.full_tokens = static_cast<int32_t>(a.full_tokens);
-  for (int r = 0; r < a.n_head; ++r) p.buf_heads[r] = a.head_start[r + 1] - a.head_start[r];
+  for (int r = 0; r < a.n_head; ++r) p.buf_heads[r] = head_units(a, r);
   int rc;
   for (int t = 0; t < a.ntensors; ++t) {
     for (int s = 0; s < a.n_seq; ++s) {
@@ -261,7 +266,7 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
         return rc;
     }
     for (int r = 0; r < a.n_head; ++r) {
-      const int64_t c = a.head_start[r + 1] - a.head_start[r];
+      const int64_t c = head_units(a, r);
       if (c == 0) continue;
       const int64_t ft = a.full_tokens;
       const bool head_major = a.head_layout == 1;  // [C][outer][full][unit], else [outer][full][C][unit]
@@ -273,13 +278,8 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
     }
   }
   const size_t smem = static_cast<size_t>(kStages) * p.stage_bytes + 128;  // + alignment of the base
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(pack_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(pack smem)");
-    configured = smem;
-  }
+  if (int rc = ensure_smem_limit(reinterpret_cast<const void*>(pack_tma_kernel), smem, "cudaFuncSetAttribute(pack smem)"))
+    return rc;
   const unsigned grid = static_cast<unsigned>(p.total_units < 0x7fffffff ? p.total_units : 0x7fffffff);
   pack_tma_kernel<<<grid, 32, smem, stream>>>(p);
   count_launch();

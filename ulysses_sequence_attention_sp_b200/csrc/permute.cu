@@ -36,10 +36,10 @@ __global__ void __launch_bounds__(kThreads, 4) permute_kernel(const __grid_const
   for (int i = threadIdx.x; i < a.nsel; i += blockDim.x) {
     const int h = a.sel_head[i];
     const int r = a.sel_rank[i];
-    s_unit[i] = h;
+    s_unit[i] = h - a.seq_unit_base;
     s_rank[i] = r;
     s_local[i] = h - a.head_start[r];
-    s_count[i] = a.head_start[r + 1] - a.head_start[r];
+    s_count[i] = head_units(a, r);
   }
   __syncthreads();
 
@@ -118,12 +118,9 @@ __global__ void __launch_bounds__(kThreads, 4) permute_kernel(const __grid_const
 }  // namespace
 
 int sm_count() {
-  static int count = 0;
-  if (count == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      count = 148;
-  }
+  int dev = 0, count = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    count = 148;
   return count;
 }
 
@@ -131,7 +128,7 @@ int launch_permute(const PermuteArgs& args, int vec_bytes, cudaStream_t stream) 
   PermuteArgs a = args;
   for (int s = 0; s < a.n_seq; ++s) a.seq_ext[s] = (a.seq_rows[s + 1] - a.seq_rows[s]) * a.heads * a.dv;
   for (int r = 0; r < a.n_head; ++r)
-    a.head_ext[r] = a.outer * a.full_tokens * (a.head_start[r + 1] - a.head_start[r]) * a.dv;
+    a.head_ext[r] = a.outer * a.full_tokens * head_units(a, r) * a.dv;
   const int64_t rows = a.seq_rows[a.n_seq];
   if (rows == 0 || a.nsel == 0) return USP_OK;
   // Work units of 4 batches (up to 512 vectors of a row), one CTA of 8 warps

@@ -12,7 +12,10 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -145,7 +148,8 @@ void select_chunk_heads(usp::PermuteArgs& a, const usp_plan* p, int lo, int hi) 
 // rank 0's shard to the others.
 int launch_pack(const usp_plan* plan, const usp::PermuteArgs& a, int vec, int64_t unit, cudaStream_t stream) {
   const bool tma = plan->pack_mode == USP_PACK_TMA && usp::pack_tma_supported(plan->elem, unit) &&
-                   a.seq_rows[a.n_seq] <= INT32_MAX && (a.dir == 0 || a.nsel == a.heads);
+                   a.seq_rows[a.n_seq] <= INT32_MAX && (a.dir == 0 || a.nsel == a.heads) &&
+                   (a.prefix == 0 || a.tok_start[0] == 0);
   if (!tma) return usp::launch_permute(a, vec, stream);
   if (int rc = usp::launch_pack_tma(a, plan->elem, unit, stream)) return rc;
   if (a.dir == 0 || a.prefix == 0 || a.n_seq < 2) return USP_OK;
@@ -223,53 +227,28 @@ int cuda_check(cudaError_t e, const char* what) {
   return set_error(USP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-}  // namespace usp
-
-extern "C" {
-
-const char* usp_last_error_message(void) { return g_last_error.c_str(); }
-
-int usp_version(void) { return 100; }
-
-int usp_balanced_ranges(int64_t total, int32_t parts, int64_t* starts, int64_t* lengths) {
-  if (!starts || !lengths) return usp::set_error(USP_ERR_INVALID_ARG, "output arrays must not be NULL");
-  return balanced(total, parts, starts, lengths);
-}
-
-int usp_seq_split(int64_t total, int32_t world, int64_t* out_counts) {
-  if (!out_counts) return usp::set_error(USP_ERR_INVALID_ARG, "out_counts is NULL");
-  return balanced(total, world, nullptr, out_counts);
-}
-
-int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_out, int32_t* lo, int32_t* hi) {
-  if (!n_out || !lo || !hi) return usp::set_error(USP_ERR_INVALID_ARG, "output pointers must not be NULL");
-  if (group_heads < 1) return usp::set_error(USP_ERR_INVALID_ARG, "group_heads must be positive");
-  if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive");
-  const int32_t size = (group_heads + num_chunks - 1) / num_chunks;
-  int32_t n = 0;
-  for (int32_t a = 0; a < group_heads; a += size, ++n) {
-    lo[n] = a;
-    hi[n] = a + size < group_heads ? a + size : group_heads;
-  }
-  *n_out = n;
+int ensure_smem_limit(const void* func, size_t bytes, const char* what) {
+  static std::mutex m;
+  static std::map<std::pair<const void*, int>, size_t> limits;
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_check(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> guard(m);
+  size_t& set = limits[{func, dev}];
+  if (bytes <= set) return USP_OK;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_check(e, what);
+  set = bytes;
   return USP_OK;
 }
 
-int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim, int32_t world,
-                    int32_t dtype, int32_t prefix_tokens) {
-  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads, head_dim, world, 1, dtype, prefix_tokens);
-}
+}  // namespace usp
 
-int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
-                        int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens) {
-  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads_kv, head_dim, world, 1, dtype, prefix_tokens);
-}
+namespace usp {
 
-int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
-                           int32_t head_dim, int32_t ulysses_size, int32_t ring_size, int32_t dtype,
-                           int32_t prefix_tokens) {
-  if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
-  *out = nullptr;
+// The plan's device-free part: sizes, the balanced token and head splits and
+// the grouped-query check. Fills *p; returns a status (the message is set).
+int plan_geometry(usp_plan* p, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv, int32_t head_dim,
+                  int32_t ulysses_size, int32_t ring_size, int32_t dtype, int32_t prefix_tokens) {
   if (ulysses_size < 1 || ring_size < 1 || static_cast<int64_t>(ulysses_size) * ring_size > USP_MAX_WORLD)
     return usp::set_error(USP_ERR_INVALID_ARG, "ulysses_size * ring_size must be in [1, %d] (got %d x %d)",
                           USP_MAX_WORLD, ulysses_size, ring_size);
@@ -282,7 +261,6 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
     return usp::set_error(USP_ERR_INVALID_ARG, "prefix_tokens must be 0 or 1 (got %d)", prefix_tokens);
   const int e = elem_bytes(dtype);
   if (!e) return usp::set_error(USP_ERR_DTYPE, "unknown dtype %d", dtype);
-  usp_plan* p = new usp_plan();
   p->batch = batch;
   p->seq_len = seq_len;
   p->heads = heads;
@@ -337,6 +315,59 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
         }
     }
   }
+  return rc;
+}
+
+}  // namespace usp
+
+extern "C" {
+
+const char* usp_last_error_message(void) { return g_last_error.c_str(); }
+
+int usp_version(void) { return 100; }
+
+int usp_balanced_ranges(int64_t total, int32_t parts, int64_t* starts, int64_t* lengths) {
+  if (!starts || !lengths) return usp::set_error(USP_ERR_INVALID_ARG, "output arrays must not be NULL");
+  return balanced(total, parts, starts, lengths);
+}
+
+int usp_seq_split(int64_t total, int32_t world, int64_t* out_counts) {
+  if (!out_counts) return usp::set_error(USP_ERR_INVALID_ARG, "out_counts is NULL");
+  return balanced(total, world, nullptr, out_counts);
+}
+
+int usp_head_chunk_ranges(int32_t group_heads, int32_t num_chunks, int32_t* n_out, int32_t* lo, int32_t* hi) {
+  if (!n_out || !lo || !hi) return usp::set_error(USP_ERR_INVALID_ARG, "output pointers must not be NULL");
+  if (group_heads < 1) return usp::set_error(USP_ERR_INVALID_ARG, "group_heads must be positive");
+  if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive");
+  const int32_t size = (group_heads + num_chunks - 1) / num_chunks;
+  int32_t n = 0;
+  for (int32_t a = 0; a < group_heads; a += size, ++n) {
+    lo[n] = a;
+    hi[n] = a + size < group_heads ? a + size : group_heads;
+  }
+  *n_out = n;
+  return USP_OK;
+}
+
+int usp_plan_create(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim, int32_t world,
+                    int32_t dtype, int32_t prefix_tokens) {
+  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads, head_dim, world, 1, dtype, prefix_tokens);
+}
+
+int usp_plan_create_gqa(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                        int32_t head_dim, int32_t world, int32_t dtype, int32_t prefix_tokens) {
+  return usp_plan_create_hybrid(out, batch, seq_len, heads, heads_kv, head_dim, world, 1, dtype, prefix_tokens);
+}
+
+int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv,
+                           int32_t head_dim, int32_t ulysses_size, int32_t ring_size, int32_t dtype,
+                           int32_t prefix_tokens) {
+  if (!out) return usp::set_error(USP_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  usp_plan* p = new usp_plan();
+  int rc = usp::plan_geometry(p, batch, seq_len, heads, heads_kv, head_dim, ulysses_size, ring_size, dtype,
+                              prefix_tokens);
   if (rc != USP_OK) {
     delete p;
     return rc;
@@ -348,7 +379,15 @@ int usp_plan_create_hybrid(usp_plan** out, int64_t batch, int64_t seq_len, int32
     return usp::set_error(USP_ERR_NO_DEVICE, "no CUDA device is visible");
   }
   cudaError_t ce = cudaGetDevice(&p->device);
-  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&p->aux, cudaStreamNonBlocking);
+  if (ce == cudaSuccess) {
+    // The allocation-free entry point's scratch address, looked up here so that
+    // the call itself never loads a module or touches the runtime's symbol table.
+    if (int src = usp::noalloc_scratch_lookup(&p->noalloc_scratch)) {
+      usp_plan_destroy(p);
+      return src;
+    }
+    ce = cudaStreamCreateWithFlags(&p->aux, cudaStreamNonBlocking);
+  }
   if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&p->ev_inputs, cudaEventDisableTiming);
   for (int c = 0; ce == cudaSuccess && c < p->group_heads; ++c) {
     cudaEvent_t ev;
@@ -738,6 +777,8 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
                                   void* workspace, size_t workspace_bytes, void* stream) {
   NvtxRange range("usp_ulysses_attention");
   if (int rc = check_plan(plan)) return rc;
+  // One call's event records, waits and launches are enqueued as a unit.
+  std::lock_guard<std::recursive_mutex> guard(plan->lock);
   if (num_chunks < 1) return usp::set_error(USP_ERR_INVALID_ARG, "num_chunks must be positive (got %d)", num_chunks);
   if (int rc = check_ptrs(q, plan->world, "q")) return rc;
   if (int rc = check_ptrs(k, plan->world, "k")) return rc;
@@ -887,6 +928,9 @@ int usp_ulysses_attention_graph_create(usp_graph** out, const usp_plan* plan, co
   if (int rc = check_plan(plan)) return rc;
   if (int rc = device_matches(plan)) return rc;
   NvtxRange range("usp_ulysses_attention_graph_create");
+  // No other call may enqueue on the plan's auxiliary stream while the capture
+  // has pulled it in.
+  std::lock_guard<std::recursive_mutex> guard(plan->lock);
   cudaStream_t cap = nullptr;
   if (int rc = usp::cuda_check(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking), "cudaStreamCreate")) return rc;
   int rc = usp::cuda_check(cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal), "cudaStreamBeginCapture");
@@ -954,6 +998,7 @@ int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas) {
 
 int usp_plan_set_timing_events(usp_plan* plan, void* start, void* stop) {
   if (int rc = check_plan(plan)) return rc;
+  std::lock_guard<std::recursive_mutex> guard(plan->lock);
   if ((start == nullptr) != (stop == nullptr))
     return usp::set_error(USP_ERR_INVALID_ARG, "set both timing events or neither");
   plan->t_start = static_cast<cudaEvent_t>(start);
@@ -997,3 +1042,25 @@ int usp_debug_wait_timeout(uint32_t limit_us, void* stream) {
 }
 
 }  // extern "C"
+
+// Helpers shared with the rank-local (multi-process) entry points in dist.cpp.
+namespace usp {
+
+int plan_vec_bytes(const usp_plan* plan) { return pick_vec(static_cast<int64_t>(plan->head_dim) * plan->elem); }
+
+int plan_launch_pack(const usp_plan* plan, const PermuteArgs& a, cudaStream_t stream) {
+  const int64_t unit = static_cast<int64_t>(plan->head_dim) * plan->elem;
+  return launch_pack(plan, a, pick_vec(unit), unit, stream);
+}
+
+int plan_check_ptr(const void* p, const char* what) { return check_ptr(p, what); }
+
+int plan_check_device(const usp_plan* plan) { return device_matches(plan); }
+
+int plan_check_attention(const usp_plan* plan) { return check_attention_shape(plan); }
+
+int plan_launch_attention(const AttnLaunch& L, cudaStream_t stream) { return launch_attention(L, stream); }
+
+float plan_scale(const usp_plan* plan, float scale) { return resolve_scale(plan, scale); }
+
+}  // namespace usp

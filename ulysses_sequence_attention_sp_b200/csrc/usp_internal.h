@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include "usp.h"
@@ -40,6 +41,15 @@ struct usp_plan {
   std::vector<cudaEvent_t> ev_chunk;      // aux -> caller stream: chunk c packed
   cudaEvent_t t_start = nullptr;          // caller-owned timing events (profiling hook)
   cudaEvent_t t_stop = nullptr;
+  // Held while one call enqueues its work (event records, waits and launches
+  // on the caller's stream and on `aux`), so that calls from several host
+  // threads never interleave their event records and waits. Recursive: the
+  // graph capture holds it around the call it captures.
+  mutable std::recursive_mutex lock;
+  // Device address of the allocation-free entry point's fixed scratch array on
+  // this plan's device, looked up when the plan is created (the plan lives no
+  // longer than the CUDA context it was created in).
+  void* noalloc_scratch = nullptr;
 
   int64_t tokens() const { return prefix + seq_len; }
 };
@@ -74,6 +84,14 @@ struct PermuteArgs {
   int32_t head_start[USP_MAX_WORLD + 1];  // head-unit range of head-side buffer r
   uint16_t sel_head[USP_MAX_HEADS];       // moved head units, ascending
   uint8_t sel_rank[USP_MAX_HEADS];        // head-side buffer owning each moved unit
+  // Optional: explicit unit counts of the head-side buffers (explicit_counts
+  // != 0), for buffers whose unit ranges leave gaps (one head chunk of every
+  // rank); otherwise buffer r holds units [head_start[r], head_start[r+1]).
+  int32_t explicit_counts;
+  // Sequence-side rows hold units [seq_unit_base, seq_unit_base + heads) of the
+  // head numbering (a row of one head chunk); 0 for whole rows.
+  int32_t seq_unit_base;
+  int32_t head_count[USP_MAX_WORLD];
   void* seq_ptr[3][USP_MAX_WORLD];
   void* head_ptr[3][USP_MAX_WORLD];
   int64_t seq_ext[USP_MAX_WORLD];   // vectors in sequence-side buffer s (set by launch_permute)
@@ -81,6 +99,11 @@ struct PermuteArgs {
 };
 
 // vec_bytes in {16, 8, 4, 2}; dv counts vectors of that size.
+// Units held by head-side buffer r.
+__host__ __device__ inline int32_t head_units(const PermuteArgs& a, int r) {
+  return a.explicit_counts ? a.head_count[r] : a.head_start[r + 1] - a.head_start[r];
+}
+
 int launch_permute(const PermuteArgs& a, int vec_bytes, cudaStream_t stream);
 
 // Bounds-checking builds: the first out-of-range site each copy kernel
@@ -99,6 +122,19 @@ int launch_pack_tma(const PermuteArgs& a, int elem, int64_t unit_bytes, cudaStre
 int read_pack_error(uint32_t* code, bool reset);
 
 int sm_count();
+
+// Raises kernel `func`'s dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is per device, so the value set is remembered
+// per (kernel, device); thread-safe.
+int ensure_smem_limit(const void* func, size_t bytes, const char* what);
+
+// The plan's device-free part (sizes, splits, grouped-query check): plan.cpp.
+int plan_geometry(usp_plan* p, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv, int32_t head_dim,
+                  int32_t ulysses_size, int32_t ring_size, int32_t dtype, int32_t prefix_tokens);
+
+// Device address of the allocation-free entry point's scratch array on the
+// current device (noalloc.cu).
+int noalloc_scratch_lookup(void** out);
 
 // ------------------------------------------------------- row collectives
 // Ragged row collectives over the plan's token split. Rank r's local buffer is
@@ -151,12 +187,12 @@ int launch_reduce_scatter_rows(const RowsArgs& a, int vec_bytes, int dtype, cuda
 // -------------------------------------------------------------- attention
 // Where output rows go. Row t of (batch b, head g): rows t < prefix go to every
 // segment; other rows go to the segment s whose token range holds t - prefix.
-// Address (elements): ptr_s + ((b * (prefix + len_s) + row_in_s) * out_heads + g) * D.
+// Address (elements): ptr_s + ((b * (prefix + len_s) + row_in_s) * out_heads + g - head_base) * D.
 struct AttnOut {
   int32_t nseg;
   int32_t prefix;
   int32_t out_heads;
-  int32_t pad0;
+  int32_t head_base;  // head coordinate g is written at head g - head_base of a segment row
   int64_t seg_start[USP_MAX_WORLD];
   int64_t seg_len[USP_MAX_WORLD];
   void* seg_ptr[USP_MAX_WORLD];
@@ -253,5 +289,14 @@ int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream);
 int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream);
 int read_attention_error(uint32_t* code, bool reset);
 int launch_wait_timeout_probe(uint32_t limit_us, cudaStream_t stream);
+
+// Plan helpers shared by the entry points of plan.cpp and dist.cpp (plan.cpp).
+int plan_vec_bytes(const usp_plan* plan);
+int plan_launch_pack(const usp_plan* plan, const PermuteArgs& a, cudaStream_t stream);
+int plan_check_ptr(const void* p, const char* what);
+int plan_check_device(const usp_plan* plan);
+int plan_check_attention(const usp_plan* plan);
+int plan_launch_attention(const AttnLaunch& L, cudaStream_t stream);
+float plan_scale(const usp_plan* plan, float scale);
 
 }  // namespace usp
