@@ -49,7 +49,6 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
     "attention": ["ulysses_sequence_attention_sp_b200/csrc/attn_tc.cu",
                   "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh"],
-    "permute": ["ulysses_sequence_attention_sp_b200/csrc/permute.cu"],
     "pack_tma": ["ulysses_sequence_attention_sp_b200/csrc/pack_tma.cu",
                  "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh"],
 }

@@ -1,5 +1,5 @@
 """The bounds-checking build (-DUSP_BOUNDS_CHECK) against the layout, row,
-ring, TMA-pack and guard-band tests.
+ring, TMA-pack, guard-band and rank-local (multi-process) tests.
 
 In that build every global offset the copy kernels and the attention
 epilogues compute is checked against its buffer's extent; an out-of-range
@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 FILES = ["tests/test_gpu_layout.py", "tests/test_gpu_rows.py", "tests/test_gpu_ring.py",
-         "tests/test_gpu_pack_tma.py", "tests/test_gpu_guard_bands.py"]
+         "tests/test_gpu_pack_tma.py", "tests/test_gpu_guard_bands.py", "tests/test_gpu_dist.py"]
 
 
 def test_checked_build_passes_the_copy_and_attention_tests():

@@ -101,6 +101,18 @@ _SIGNATURES = {
     "usp_ulysses_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, _c_vpp, _c_vpp, _c_vpp, _c_vpp, ctypes.c_float,
                                                      ctypes.c_int32, ctypes.c_void_p]),
     "usp_plan_set_timing_events": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "usp_dist_exchange_counts": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                _c_i64p, _c_i64p, _c_i64p, _c_i64p]),
+    "usp_dist_pack": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, _c_vpp, ctypes.c_void_p, ctypes.c_void_p]),
+    "usp_dist_unpack": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, _c_vpp, ctypes.c_void_p]),
+    "usp_dist_workspace_size": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
+    "usp_dist_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "usp_kernel_launches": (ctypes.c_uint64, []),
     "usp_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "usp_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_void_p]),
@@ -546,6 +558,77 @@ def ulysses_attention_noalloc(plan: Plan, q, k, v, out=None, scale: float = 0.0,
     _check(_lib.usp_ulysses_attention_noalloc(plan.handle, _ptrs(q), _ptrs(k), _ptrs(v), _ptrs(out), float(scale),
                                               num_chunks, _stream(stream)))
     return out
+
+
+# ------------------------------------------- rank-local (multi-process) steps
+# One process per GPU and per sequence-parallel rank: the library packs,
+# unpacks and computes; the exchange itself is the caller's collective (the
+# `dist` module runs it over torch.distributed). Wire format: include/usp.h.
+DIST_SEQ_TO_HEAD, DIST_HEAD_TO_SEQ, DIST_GATHER_SEQ, DIST_GATHER_HEADS = 0, 1, 2, 3
+
+
+def dist_exchange_counts(batch: int, seq_len: int, heads: int, head_dim: int, world: int, rank: int, exchange: int,
+                         ntensors: int = 1, num_chunks: int = 1, chunk: int = 0, prefix: int = 0,
+                         kv_heads: int | None = None):
+    """Transport page, seq_to_heads' split lists for one exchange of `rank`, in
+    elements: (send_counts, send_displs, recv_counts, recv_displs). Needs no
+    device."""
+    arrs = [(ctypes.c_int64 * max(int(world), 1))() for _ in range(4)]
+    _check(_lib.usp_dist_exchange_counts(batch, seq_len, heads, heads if kv_heads is None else kv_heads, head_dim,
+                                         world, prefix, rank, exchange, ntensors, num_chunks, chunk, *arrs))
+    return tuple([a[i] for i in range(world)] for a in arrs)
+
+
+def dist_counts(plan: Plan, rank: int, exchange: int, ntensors: int = 1, num_chunks: int = 1, chunk: int = 0):
+    """dist_exchange_counts for a plan's sizes."""
+    return dist_exchange_counts(plan.batch, plan.seq_len, plan.heads, plan.head_dim, plan.world, rank, exchange,
+                                ntensors, num_chunks, chunk, plan.prefix, plan.kv_heads)
+
+
+def _flat_buffer(t, plan: Plan, what: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise UspError(USP_ERR_INVALID_ARG, f"{what} must be a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def dist_pack(plan: Plan, rank: int, exchange: int, tensors, send, num_chunks: int = 1, chunk: int = 0,
+              stream=None):
+    """Fills the flat `send` buffer of one exchange from this rank's tensors
+    (sequence shards of q[, k, v], or its head shard o)."""
+    n = len(tensors)
+    _check_tensors(plan, list(tensors), [None] * n, "in")
+    _check(_lib.usp_dist_pack(plan.handle, rank, exchange, n, num_chunks, chunk, _ptrs(tensors),
+                              _flat_buffer(send, plan, "send"), _stream(stream)))
+    return send
+
+
+def dist_unpack(plan: Plan, rank: int, exchange: int, recv, out, num_chunks: int = 1, chunk: int = 0,
+                stream=None):
+    """Reads the flat `recv` buffer of one exchange into this rank's tensors
+    (head shards of q[, k, v], or its sequence shard)."""
+    n = len(out)
+    _check_tensors(plan, list(out), [None] * n, "out")
+    _check(_lib.usp_dist_unpack(plan.handle, rank, exchange, n, num_chunks, chunk, _flat_buffer(recv, plan, "recv"),
+                                _ptrs(out), _stream(stream)))
+    return out
+
+
+def dist_workspace_bytes(plan: Plan, rank: int) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.usp_dist_workspace_size(plan.handle, rank, ctypes.byref(n)))
+    return n.value
+
+
+def dist_attention(plan: Plan, rank: int, exchange: int, recv, send_o, workspace, num_chunks: int = 1,
+                   chunk: int = 0, scale: float = 0.0, stream=None):
+    """Attention of one head chunk on this rank: received q/k/v (`exchange`
+    SEQ_TO_HEAD or GATHER_SEQ) in, the output written into `send_o` in the
+    layout of the way back (HEAD_TO_SEQ or GATHER_HEADS)."""
+    _check(_lib.usp_dist_attention(plan.handle, rank, exchange, num_chunks, chunk, _flat_buffer(recv, plan, "recv"),
+                                   _flat_buffer(send_o, plan, "send_o"), float(scale),
+                                   _flat_buffer(workspace, plan, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+    return send_o
 
 
 def kernel_launches() -> int:
