@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--no-reshard", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads (measured after the headline, 1 GPU only)")
+    ap.add_argument("--attention-kernel", choices=["auto", "one_tile", "two_tile"], default="auto",
+                    help="the tensor-core attention kernel (all compute the same function)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying the step as one CUDA graph")
     return ap.parse_args()
@@ -271,10 +273,12 @@ class BlockBench:
     in L2 get a 512 MiB write between timed steps, whose time is measured apart
     and subtracted."""
 
-    def __init__(self, usp, torch, dev, w, n_chunks, steps, seed, graph=True):
+    def __init__(self, usp, torch, dev, w, n_chunks, steps, seed, graph=True, kernel="auto"):
         self.usp, self.torch, self.dev, self.w, self.n_chunks, self.steps = usp, torch, dev, w, n_chunks, steps
         self.plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix,
                              kv_heads=w.heads_kv, ring_size=w.ring)
+        if kernel != "auto" and w.dtype != "fp32":
+            self.plan.set_attention_kernel(kernel)
         plan = self.plan
         self.storage = make_qkv(w, seed=seed)
         self.full = [self.to_dev(x) for x in self.storage]
@@ -462,7 +466,8 @@ def run_ours(args, w, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    bb = BlockBench(usp, torch, dev, w, n_chunks, args.steps, seed=w.seed + 7919 * rank, graph=not args.no_graph)
+    bb = BlockBench(usp, torch, dev, w, n_chunks, args.steps, seed=w.seed + 7919 * rank, graph=not args.no_graph,
+                    kernel=args.attention_kernel)
     bb.prepare(args.warmup)
     # timed region: exactly K steps, attention kernels bracketed by their own events
     clocks = ClockSampler(local_rank)
@@ -490,7 +495,8 @@ def run_ours(args, w, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {**workload_config(w, n_chunks, world), "cuda_graph": bool(bb.graphs)},
+            "config": {**workload_config(w, n_chunks, world), "cuda_graph": bool(bb.graphs),
+                   "attention_kernel": args.attention_kernel},
             "roofline": roof,
             "gpu_launches": int(launches),
             "clocks": clk,

@@ -195,6 +195,26 @@ int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode);
  */
 int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas);
 
+/*
+ * usp_plan_set_attention_kernel -- which tensor-core attention kernel this
+ * plan's 16-bit attention launches use (all compute the same function; see
+ * usp_head_attention). USP_ATTN_ONE_TILE: one 128-row query tile per CTA with
+ * 256-key tiles and four softmax threads per row (persistent CTAs for short
+ * key sequences or under a CTA cap). USP_ATTN_TWO_TILE: two 128-row query
+ * tiles per CTA with 128-key tiles and one softmax thread per row, the two
+ * tiles' softmax and tensor-core work interleaved; head_dim a multiple of 16
+ * in [64, 128]. USP_ATTN_AUTO (the default): TWO_TILE where it applies and the
+ * launch has more than 16 key tiles of 256 and no CTA cap, ONE_TILE
+ * otherwise. Results agree within rounding (the tile sizes differ, so the
+ * order of the fp32 sums differs). The fp32 path ignores it. Errors:
+ * USP_ERR_INVALID_ARG for an unknown value, USP_ERR_UNSUPPORTED for TWO_TILE
+ * with another dtype or head_dim.
+ */
+#define USP_ATTN_AUTO 0
+#define USP_ATTN_ONE_TILE 1
+#define USP_ATTN_TWO_TILE 2
+int usp_plan_set_attention_kernel(usp_plan* plan, int32_t kernel);
+
 /* Copies the plan's Ulysses group size and ring size out (world and 1 for a plain plan); either may be NULL. */
 int usp_plan_query_hybrid(const usp_plan* plan, int32_t* ulysses_size, int32_t* ring_size);
 

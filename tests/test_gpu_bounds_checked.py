@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 FILES = ["tests/test_gpu_layout.py", "tests/test_gpu_rows.py", "tests/test_gpu_ring.py",
-         "tests/test_gpu_pack_tma.py", "tests/test_gpu_guard_bands.py", "tests/test_gpu_dist.py"]
+         "tests/test_gpu_pack_tma.py", "tests/test_gpu_guard_bands.py", "tests/test_gpu_dist.py",
+         "tests/test_gpu_two_tile.py"]
 
 
 def test_checked_build_passes_the_copy_and_attention_tests():

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libusp.so")
 # through $USP_LIBRARY.
 CHECKED_LIB_PATH = os.path.join(PKG_DIR, "libusp_checked.so")
 
-SOURCES = ["plan.cpp", "tensor_map.cpp", "permute.cu", "pack_tma.cu", "rows.cu", "attn_tc.cu", "attn_simt.cu", "noalloc.cu", "dist.cpp"]
+SOURCES = ["plan.cpp", "tensor_map.cpp", "permute.cu", "pack_tma.cu", "rows.cu", "attn_tc.cu", "attn_pp.cu", "attn_simt.cu", "noalloc.cu", "dist.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           f"-I{INCLUDE}", f"-I{CSRC}"]

@@ -495,6 +495,7 @@ int usp_dist_attention(const usp_plan* plan, int32_t rank, int32_t exchange, int
   L.dtype = p->dtype;
   L.scale = usp::plan_scale(p, scale);
   L.max_ctas = p->attn_ctas;
+  L.kernel = p->attn_kernel;
   L.n_heads = own.nq;
   for (int i = 0; i < own.nq; ++i) L.heads[i] = static_cast<uint16_t>(x.lo + i);
   return usp::plan_launch_attention(L, s);

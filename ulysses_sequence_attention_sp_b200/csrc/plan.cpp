@@ -702,6 +702,7 @@ int usp_head_attention(const usp_plan* plan, const void* const* q_heads, const v
     L.dtype = plan->dtype;
     L.scale = resolve_scale(plan, scale);
     L.max_ctas = plan->attn_ctas;
+    L.kernel = plan->attn_kernel;
     for (int h = 0; h < hr; ++h) L.heads[h] = static_cast<uint16_t>(h);
     if (int rc = launch_attention(L, s)) return rc;
   }
@@ -870,6 +871,7 @@ static int ulysses_attention_impl(const usp_plan* plan, const void* const* q, co
   L.dtype = plan->dtype;
   L.scale = resolve_scale(plan, scale);
   L.max_ctas = plan->attn_ctas;
+  L.kernel = plan->attn_kernel;
   L.lse = lse;
   if (plan->ring > 1) {
     // Ring: query group g = key block g = token block of Ulysses group g
@@ -996,6 +998,18 @@ int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas) {
   return USP_OK;
 }
 
+int usp_plan_set_attention_kernel(usp_plan* plan, int32_t kernel) {
+  if (int rc = check_plan(plan)) return rc;
+  if (kernel != USP_ATTN_AUTO && kernel != USP_ATTN_ONE_TILE && kernel != USP_ATTN_TWO_TILE)
+    return usp::set_error(USP_ERR_INVALID_ARG, "unknown attention kernel %d", kernel);
+  if (kernel == USP_ATTN_TWO_TILE && !usp::attention_pp_supported(plan->dtype, plan->head_dim))
+    return usp::set_error(USP_ERR_UNSUPPORTED, "the two-query-tile kernel takes 16-bit inputs with head_dim a "
+                          "multiple of 16 in [64, 128] (got dtype %d, head_dim %d)", plan->dtype, plan->head_dim);
+  std::lock_guard<std::recursive_mutex> guard(plan->lock);
+  plan->attn_kernel = kernel;
+  return USP_OK;
+}
+
 int usp_plan_set_timing_events(usp_plan* plan, void* start, void* stop) {
   if (int rc = check_plan(plan)) return rc;
   std::lock_guard<std::recursive_mutex> guard(plan->lock);
@@ -1013,9 +1027,11 @@ int usp_device_status(uint32_t* code, int32_t reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return usp::cuda_check(e, "cudaDeviceSynchronize");
   if (int rc = usp::read_attention_error(code, reset != 0)) return rc;
-  uint32_t pack_code = 0;
+  uint32_t pack_code = 0, pp_code = 0;
   if (int rc = usp::read_pack_error(&pack_code, reset != 0)) return rc;
+  if (int rc = usp::read_pp_error(&pp_code, reset != 0)) return rc;
   if (*code == 0) *code = pack_code;
+  if (*code == 0) *code = pp_code;
   if (*code != 0) {
     usp::set_error(USP_ERR_TIMEOUT, "a device-side wait ran out (site %u)", *code);
     return USP_ERR_TIMEOUT;
@@ -1023,7 +1039,7 @@ int usp_device_status(uint32_t* code, int32_t reset) {
   // Bounds-checking builds record the first out-of-range access per kernel file.
   int (*const readers[])(uint32_t*, bool) = {usp::read_permute_bounds, usp::read_rows_bounds,
                                              usp::read_pack_bounds, usp::read_attention_bounds,
-                                             usp::read_simt_bounds};
+                                             usp::read_simt_bounds, usp::read_pp_bounds};
   for (auto read : readers) {
     uint32_t site = 0;
     if (int rc = read(&site, reset != 0)) return rc;

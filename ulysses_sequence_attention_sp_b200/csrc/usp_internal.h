@@ -35,6 +35,7 @@ struct usp_plan {
   int32_t ring = 1;
   int32_t pack_mode = USP_PACK_TMA;  // USP_PACK_TMA (default) or USP_PACK_VECTOR: how seq->head packs move data
   int32_t attn_ctas = 0;  // cap on the attention kernel's CTAs (0: automatic)
+  int32_t attn_kernel = USP_ATTN_AUTO;  // which tensor-core attention kernel (usp_plan_set_attention_kernel)
   int device = 0;
   cudaStream_t aux = nullptr;             // runs the per-chunk seq->head packs
   cudaEvent_t ev_inputs = nullptr;        // caller stream -> aux: inputs ready
@@ -248,6 +249,7 @@ struct AttnLaunch {
   int32_t dtype;
   float scale;
   int32_t max_ctas;  // cap on the tensor-core kernel's CTAs (0: automatic)
+  int32_t kernel;    // USP_ATTN_AUTO, USP_ATTN_ONE_TILE or USP_ATTN_TWO_TILE
   uint16_t heads[USP_MAX_HEADS];
 };
 
@@ -285,6 +287,11 @@ int make_map(CUtensorMap* map, const void* base, const AttnView& view, const Att
              int box_rows);
 
 bool attention_tc_supported(int dtype, int head_dim);
+// Two query tiles per CTA (attn_pp.cu): 16-bit, head_dim 64..128 in steps of 16.
+bool attention_pp_supported(int dtype, int head_dim);
+int launch_attention_pp(const AttnLaunch& L, cudaStream_t stream);
+int read_pp_error(uint32_t* code, bool reset);
+int read_pp_bounds(uint32_t* code, bool reset);
 int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream);
 int launch_attention_simt(const AttnLaunch& L, cudaStream_t stream);
 int read_attention_error(uint32_t* code, bool reset);

@@ -75,6 +75,7 @@ _SIGNATURES = {
                                                  ctypes.c_void_p]),
     "usp_plan_set_pack_mode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
     "usp_plan_set_attention_ctas": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
+    "usp_plan_set_attention_kernel": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32]),
     "usp_ulysses_attention_graph_create": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p, _c_vpp,
                                                           _c_vpp, _c_vpp, _c_vpp, ctypes.c_float, ctypes.c_int32,
                                                           ctypes.c_void_p, ctypes.c_size_t]),
@@ -287,6 +288,15 @@ class Plan:
         fewer CTAs than (query tile, batch, head) items each CTA walks several."""
         _check(_lib.usp_plan_set_attention_ctas(self.handle, int(max_ctas)))
         self.attention_ctas = int(max_ctas)
+
+    def set_attention_kernel(self, kernel: str) -> None:
+        """'auto' (default), 'one_tile' or 'two_tile': which tensor-core
+        attention kernel runs (same function; see include/usp.h)."""
+        codes = {"auto": 0, "one_tile": 1, "two_tile": 2}
+        if kernel not in codes:
+            raise UspError(USP_ERR_INVALID_ARG, f"attention kernel must be one of {sorted(codes)}")
+        _check(_lib.usp_plan_set_attention_kernel(self.handle, codes[kernel]))
+        self.attention_kernel = kernel
 
     def workspace_bytes(self, num_chunks: int = 1) -> int:
         n = ctypes.c_size_t()
