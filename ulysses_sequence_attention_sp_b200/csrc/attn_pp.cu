@@ -41,6 +41,21 @@ namespace usp {
 __device__ uint32_t g_pp_error;   // first wait that ran out (site code), 0 if none
 __device__ uint32_t g_pp_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
 
+// Pipeline trace (built only with -DUSP_TRACE): clock64() at pipeline events
+// of CTA 7, [event][key tile]; read with usp_debug_read_trace_pp.
+#ifdef USP_TRACE
+constexpr int kPpTraceEvents = 16, kPpTraceTiles = 256;
+__device__ unsigned long long g_pp_trace[kPpTraceEvents][kPpTraceTiles];
+#define PP_TRACE(ev, j)                                                                   \
+  do {                                                                                    \
+    if (blockIdx.x == 7 && blockIdx.y == 0 && (j) < kPpTraceTiles) g_pp_trace[(ev)][(j)] = clock64(); \
+  } while (0)
+#else
+#define PP_TRACE(ev, j) \
+  do {                  \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kRows = 128;                          // query rows per tile = TMEM lanes
@@ -259,6 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, &g_pp_error, 42, kWaitLimitNs);
       tc_fence_after();
       // S_t = Q_t K^T for the K tile in ring stage st (already landed).
+#ifdef USP_TRACE
+      int s_count[2] = {0, 0};
+#endif
       auto issue_s = [&](int t, int st) {
 #pragma unroll
         for (int a = 0; a < C::NATOM; ++a)
@@ -271,10 +289,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
             umma_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, (a > 0 || ks > 0) ? 1u : 0u);
           }
         umma_commit(&bars->s_full[t]);
+#ifdef USP_TRACE
+        const int si = s_count[t]++;
+        PP_TRACE(t, si);
+#endif
       };
       // O_t += P_t(j) V_j once the softmax of tile t has stored P_t(j) (V stage st landed).
       auto issue_pv = [&](int t, int j, int st) -> bool {
         if (!mbar_wait(&bars->p_full[t], j & 1, abort_flag, &g_pp_error, 43 + t, kWaitLimitNs)) return false;
+        PP_TRACE(2 + t, j);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
@@ -354,11 +377,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
         ok = false;
         break;
       }
+      const bool tr0 = (warp & 3) == 0 && lane == 0;
+      if (tr0) PP_TRACE(4 + 5 * t, j);
       tc_fence_after();
       uint32_t sr[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys; c += 32) tmem_ld32(sc + c, sr + c);
       tmem_wait_ld();
+      if (tr0) PP_TRACE(5 + 5 * t, j);
       float* s = reinterpret_cast<float*>(sr);
       const int valid = RING ? kb_left : T - j * kKeys;  // valid keys of this tile (>= kKeys: all)
       if (valid < kKeys) {
@@ -366,17 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
         for (int c = 0; c < kKeys; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      // Row maximum: four independent three-input chains, then a tree.
-      float mx4[4];
+      // Row maximum: eight independent three-input chains, then a tree.
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float a = fmaxf(s[i], s[i + 4]);
+      for (int i = 0; i < 8; ++i) {
+        float a = fmaxf(s[i], s[i + 8]);
 #pragma unroll
-        for (int c = i + 8; c < kKeys; c += 8) a = max3(a, s[c], s[c + 4]);
-        mx4[i] = a;
+        for (int c = i + 16; c < kKeys; c += 16) a = max3(a, s[c], s[c + 8]);
+        mx8[i] = a;
       }
-      const float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+      const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m, mx * sl2);
+      if (tr0) PP_TRACE(6 + 5 * t, j);
       if (j == 0) {
         m = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
@@ -400,8 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       // first 64 columns of S (already in registers) in two halves. Masked
       // entries (s = -inf) give exactly 0.
       // The scaling and the row sum run on packed fp32 pairs (one instruction
-      // per two values). (Rounding P on the integer pipe instead of cvt, to
-      // relieve the conversion unit, measured 10% slower.)
+      // per two values). Measured and not kept: rounding P on the integer pipe
+      // instead of cvt (10% slower); a quarter or half of the exponentials as a
+      // degree-3 polynomial on the FMA pipe (4-5% slower).
       const uint64_t scale2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m, -m);
       uint64_t acc2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -425,9 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       f2_unpack(acc2[2], a4, a5);
       f2_unpack(acc2[3], a6, a7);
       l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+      if (tr0) PP_TRACE(7 + 5 * t, j);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[t]);
+      if (tr0) PP_TRACE(8 + 5 * t, j);
       if constexpr (RING) {
         kb_left -= kKeys;
         if (kb_left <= 0) {
@@ -574,6 +604,14 @@ int read_pp_error(uint32_t* code, bool reset) {
   }
   return USP_OK;
 }
+
+#ifdef USP_TRACE
+extern "C" int usp_debug_read_trace_pp(unsigned long long* out, int n) {
+  const int total = kPpTraceEvents * kPpTraceTiles;
+  if (n > total) n = total;
+  return cudaMemcpyFromSymbol(out, g_pp_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 5;
+}
+#endif
 
 int read_pp_bounds(uint32_t* code, bool reset) {
   cudaError_t e = cudaMemcpyFromSymbol(code, g_pp_bounds, sizeof(uint32_t));
