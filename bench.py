@@ -47,7 +47,7 @@ WORKLOADS = {"tiny": W.TINY, "reshard": W.RESHARD, "video": W.VIDEO, "vit": W.VI
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
-    "attention": ["ulysses_sequence_attention_sp_b200/csrc/attn_tc.cu",
+    "attention": ["ulysses_sequence_attention_sp_b200/csrc/attn_pp.cu",
                   "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh"],
     "pack_tma": ["ulysses_sequence_attention_sp_b200/csrc/pack_tma.cu",
                  "ulysses_sequence_attention_sp_b200/csrc/device_common.cuh"],
@@ -487,7 +487,7 @@ def run_ours(args, w, rank, world, local_rank):
         roof = attention_roofline(w, attn_ms_max, n_launch_attn, pk, pk_kind)
         # algorithmic bytes of one launch: q, k, v read once and o written once
         roof["traffic"] = recorded_traffic("attention", 4 * w.tensor_bytes / n_launch_attn)
-        roof["kernel"] = "attn_tc_kernel (tcgen05), one launch per head chunk"
+        roof["kernel"] = "attn_pp_kernel (tcgen05, two query tiles per CTA), one launch per head chunk"
         roof["peak_source"] += "; the kernel runs inside a long step loop"
         roof = {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "kernel",
                                      "peak_source", "frac_of_burst_peak", "attention_ms_per_step", "launch_ms")}
