@@ -67,7 +67,7 @@ def parse_args():
     ap.add_argument("--no-reshard", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads (measured after the headline, 1 GPU only)")
-    ap.add_argument("--attention-kernel", choices=["auto", "one_tile", "two_tile"], default="auto",
+    ap.add_argument("--attention-kernel", choices=["auto", "one_tile", "two_tile", "two_cta"], default="auto",
                     help="the tensor-core attention kernel (all compute the same function)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying the step as one CUDA graph")

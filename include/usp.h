@@ -203,16 +203,22 @@ int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas);
  * key sequences or under a CTA cap). USP_ATTN_TWO_TILE: two 128-row query
  * tiles per CTA with 128-key tiles and one softmax thread per row, the two
  * tiles' softmax and tensor-core work interleaved; head_dim a multiple of 16
- * in [64, 128]. USP_ATTN_AUTO (the default): TWO_TILE where it applies and the
- * launch has more than 16 key tiles of 256 and no CTA cap, ONE_TILE
- * otherwise. Results agree within rounding (the tile sizes differ, so the
- * order of the fp32 sums differs). The fp32 path ignores it. Errors:
+ * in [64, 128]. USP_ATTN_TWO_CTA: the same kernel with one 128-row query tile
+ * per CTA and two CTAs per SM, whose work the SM interleaves; head_dim 64 or
+ * 80 (the two CTAs' K and V rings must fit in one SM's shared memory).
+ * USP_ATTN_AUTO (the default), for launches without a CTA cap: TWO_TILE
+ * where it applies and the launch has more than 16 key tiles of 256; with
+ * fewer, TWO_CTA where it applies; ONE_TILE otherwise (and under a cap).
+ * Results agree within rounding (the tile sizes differ, so the order of the
+ * fp32 sums differs; TWO_TILE and TWO_CTA agree bit for bit). The fp32 path
+ * ignores it. Errors:
  * USP_ERR_INVALID_ARG for an unknown value, USP_ERR_UNSUPPORTED for TWO_TILE
- * with another dtype or head_dim.
+ * or TWO_CTA with another dtype or head_dim.
  */
 #define USP_ATTN_AUTO 0
 #define USP_ATTN_ONE_TILE 1
 #define USP_ATTN_TWO_TILE 2
+#define USP_ATTN_TWO_CTA 3
 int usp_plan_set_attention_kernel(usp_plan* plan, int32_t kernel);
 
 /* Copies the plan's Ulysses group size and ring size out (world and 1 for a plain plan); either may be NULL. */

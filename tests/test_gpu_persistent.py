@@ -1,10 +1,11 @@
-"""Persistent attention CTAs: with fewer CTAs than (query tile, batch, head)
-items, each CTA walks several items and overlaps one item's loads and first
-Q K^T with the previous item's last key tiles. Every item is computed the same
-way, so a capped launch must give the same bits as the default launch (which
-the other attention tests pin to the float64 oracle). The ViT workload, whose
-577-token items make the automatic launch persistent, is also compared with
-the oracle directly."""
+"""Persistent attention CTAs of the one-tile kernel: with fewer CTAs than
+(query tile, batch, head) items, each CTA walks several items and overlaps one
+item's loads and first Q K^T with the previous item's last key tiles. Every
+item is computed the same way, so a capped launch must give the same bits as
+the one-CTA-per-item launch of that kernel (which the other attention tests
+pin to the float64 oracle). The ViT workload (577-token items) is also
+compared with the oracle directly, through the automatic choice and through
+the persistent launch."""
 
 import numpy as np
 import pytest
@@ -42,9 +43,10 @@ def _storage(w):
     return tuple(rng.standard_normal(shape, dtype=np.float32).astype(np.float16) for _ in range(3))
 
 
-def _block(usp, w, storage, ring=1, ctas=0, num_chunks=1, lse=None):
+def _block(usp, w, storage, ring=1, ctas=0, num_chunks=1, lse=None, kernel="one_tile"):
     plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix, kv_heads=w.heads_kv,
                     ring_size=ring)
+    plan.set_attention_kernel(kernel)
     plan.set_attention_ctas(ctas)
     shards = [usp.scatter_sequence(plan, _dev(x, w)) for x in storage]
     out = plan.empty_seq_shards(fill=float("nan"))
@@ -104,18 +106,21 @@ def test_capped_lse_is_bit_identical(usp):
 
 
 def test_vit_workload_persistent_against_oracle(usp):
-    """B=16, cls + 576 patches, H=16, D=80, P=4: 1280 items of 3 key tiles,
-    so the automatic launch is persistent (one CTA per SM)."""
+    """B=16, cls + 576 patches, H=16, D=80, P=4: 1280 items of 3 key tiles of
+    256. The automatic launch (the 128-key kernel, two CTAs per SM) and the
+    persistent one-tile launch (one CTA per SM) are both compared with the
+    oracle; the persistent launch also with the one-CTA-per-item launch."""
     w = VIT
     storage = make_qkv(w)
-    bits, out, tr = _block(usp, w, storage)
-    full = np.concatenate([to_f64(o, w.dtype)[:, (w.prefix if r else 0):] for r, o in enumerate(out)], axis=1)
     ref = attention_bshd(*(storage_to_f64(x, w.dtype) for x in storage))
-    assert_close(full, ref, w.dtype, "vit")
-    # every rank's copy of the cls row is the same row
-    for o in out[1:]:
-        assert torch.equal(o[:, 0].view(torch.int16), out[0][:, 0].view(torch.int16))
-    # and the one-CTA-per-item launch gives the same bits
+    for kernel, ctas in (("auto", 0), ("one_tile", 148)):
+        bits, out, tr = _block(usp, w, storage, ctas=ctas, kernel=kernel)
+        full = np.concatenate([to_f64(o, w.dtype)[:, (w.prefix if r else 0):] for r, o in enumerate(out)], axis=1)
+        assert_close(full, ref, w.dtype, f"vit {kernel}")
+        # every rank's copy of the cls row is the same row
+        for o in out[1:]:
+            assert torch.equal(o[:, 0].view(torch.int16), out[0][:, 0].view(torch.int16))
+    # the one-CTA-per-item launch gives the persistent launch's bits
     got, _, _ = _block(usp, w, storage, ctas=1 << 30)
     for a, b in zip(got, bits):
         assert torch.equal(a, b)

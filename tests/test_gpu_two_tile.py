@@ -137,6 +137,49 @@ def test_two_tile_ring_matches_oracle(usp, case):
         plan.close()
 
 
+TWO_CTA_CASES = [w for w in CASES if w.head_dim in (64, 80)] + [
+    Workload("tc-bf16-B3-T576-cls-H4-D80-P4", 3, 576, 1, 4, 80, 4, "bf16", 1.0, 9521, (1, 2)),
+    Workload("tc-fp16-T300-H2-D64-P2", 1, 300, 0, 2, 64, 2, "fp16", 1.0, 9522, (1,)),
+]
+
+
+@pytest.mark.parametrize("w", TWO_CTA_CASES, ids=lambda w: w.name)
+def test_two_cta_matches_oracle(usp, w):
+    """One query tile per CTA, two CTAs per SM: the same kernel at QT=1."""
+    for n in w.num_chunks:
+        storage, plan, out = _run(usp, w, "two_cta", n)
+        f64 = [_f64(x, w) for x in storage]
+        sh = [ol.scatter_sequence(x, plan.token_ranges, prefix=w.prefix) for x in f64]
+        ref = oa.ulysses_attention(*sh, plan.token_ranges, plan.head_ranges, kv_head_ranges=plan.kv_head_ranges,
+                                   prefix=w.prefix)
+        for r in range(plan.world):
+            assert_close(_out64(out[r], w), ref[r], "bf16", f"{w.name} chunks={n} rank={r}")
+        plan.close()
+
+
+@pytest.mark.parametrize("case", [c for c in RING_CASES if c[0].head_dim in (64, 80)], ids=lambda c: c[0].name)
+def test_two_cta_ring_matches_oracle(usp, case):
+    w, ring = case
+    storage, plan, out = _run(usp, w, "two_cta", 1, ring=ring)
+    tr = plan.token_ranges
+    qs, ks, vs = (ol.scatter_sequence(_f64(x, w), tr, prefix=w.prefix) for x in storage)
+    ref = oring.ulysses_ring_attention(qs, ks, vs, tr, w.world // ring, ring, prefix=w.prefix)
+    for r in range(plan.world):
+        assert_close(_out64(out[r], w), ref[r], "bf16", f"{w.name} rank={r}")
+    plan.close()
+
+
+def test_two_cta_agrees_bitwise_with_two_tile(usp):
+    """Both run the same per-tile arithmetic in the same order: identical bits."""
+    w = TWO_CTA_CASES[0]
+    _, p1, o1 = _run(usp, w, "two_cta", 1)
+    _, p2, o2 = _run(usp, w, "two_tile", 1)
+    for r in range(p1.world):
+        assert torch.equal(o1[r].view(torch.int16).cpu(), o2[r].view(torch.int16).cpu()), f"rank {r}"
+    p1.close()
+    p2.close()
+
+
 def test_two_tile_lse(usp):
     w = CASES[1]
     lse = torch.full((w.heads, w.batch, w.tokens), float("nan"), dtype=torch.float32, device="cuda")
@@ -157,6 +200,14 @@ def test_two_tile_refused_where_not_built(usp):
     plan = usp.Plan(1, 100, 4, 48, 2, "bf16", 0)
     with pytest.raises(usp.UspError) as e:
         plan.set_attention_kernel("two_tile")
+    assert e.value.code == usp.USP_ERR_UNSUPPORTED
+    with pytest.raises(usp.UspError) as e:
+        plan.set_attention_kernel("two_cta")
+    assert e.value.code == usp.USP_ERR_UNSUPPORTED
+    plan.close()
+    plan = usp.Plan(1, 100, 4, 128, 2, "bf16", 0)
+    with pytest.raises(usp.UspError) as e:
+        plan.set_attention_kernel("two_cta")
     assert e.value.code == usp.USP_ERR_UNSUPPORTED
     with pytest.raises(usp.UspError) as e:
         plan.set_attention_kernel("fastest")

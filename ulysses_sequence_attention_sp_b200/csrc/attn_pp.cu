@@ -59,22 +59,21 @@ __device__ unsigned long long g_pp_trace[kPpTraceEvents][kPpTraceTiles];
 namespace {
 
 constexpr int kRows = 128;                          // query rows per tile = TMEM lanes
-constexpr int kQTiles = 2;                          // query tiles per CTA
+constexpr int kMaxQTiles = 2;                       // query tiles per CTA: QT = 2 (one CTA per SM) or 1 (two)
 constexpr int kKeys = 128;                          // keys per key tile
-constexpr int kSoftmaxWarps = 4 * kQTiles;
-constexpr int kProducerWarp = kSoftmaxWarps;
-constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
-constexpr uint32_t kTmemCols = 512;
+__host__ __device__ constexpr int pp_threads(int qt) { return 32 * (4 * qt + 2); }  // softmax, producer, MMA warps
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: only a broken pipeline waits this long
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s to let in-flight copies land on abort
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 constexpr int kMaxStages = 3;
 
+// TMEM columns of tile t's S and O when a CTA holds QT tiles.
+template <int QT>
 __device__ __forceinline__ uint32_t col_s(int t) { return static_cast<uint32_t>(t) * 128u; }
-__device__ __forceinline__ uint32_t col_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
+template <int QT>
+__device__ __forceinline__ uint32_t col_o(int t) { return 128u * QT + static_cast<uint32_t>(t) * 128u; }
 
-template <int D>
+template <int D, int QT>
 struct PpCfg {
   static constexpr int ATOM = (D % 64 == 0) ? 64 : ((D % 32 == 0) ? 32 : 16);  // elements per swizzle row
   static constexpr int NATOM = D / ATOM;
@@ -84,8 +83,11 @@ struct PpCfg {
   static constexpr int BLOCK_BYTES = 128 * ROWB;         // one atom-column block of a 128-row tile
   static constexpr int TILE_BYTES = 128 * D * 2;         // a Q, K or V tile: NATOM blocks
   static constexpr int KSTEPS = ATOM / 16;
-  static constexpr int FIXED = kQTiles * TILE_BYTES + 1024 + 2048;  // Q tiles, base alignment, barriers
-  static constexpr int STAGES = FIXED + 6 * TILE_BYTES <= 232448 ? 3 : 2;  // K and V ring depth
+  static constexpr int FIXED = QT * TILE_BYTES + 1024 + 2048;  // Q tiles, base alignment, barriers
+  // Shared memory per CTA: all of it (227 KB) for one CTA per SM; for two,
+  // half of the SM's 228 KB less the 1 KB the hardware reserves per CTA.
+  static constexpr int BUDGET = QT == 2 ? 232448 : 115712;
+  static constexpr int STAGES = FIXED + 6 * TILE_BYTES <= BUDGET ? 3 : 2;  // K and V ring depth
   static constexpr int SMEM_BYTES = FIXED + 2 * STAGES * TILE_BYTES;
 };
 
@@ -93,7 +95,7 @@ struct PpBars {
   uint64_t q_full;
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-  uint64_t s_full[kQTiles], p_full[kQTiles], o_full[kQTiles];
+  uint64_t s_full[kMaxQTiles], p_full[kMaxQTiles], o_full[kMaxQTiles];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -139,13 +141,16 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return bf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
 
-template <int D, bool BF16, bool RING>
-__global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_constant__ PpParams p) {
-  using C = PpCfg<D>;
+template <int D, int QT, bool BF16, bool RING>
+__global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const __grid_constant__ PpParams p) {
+  using C = PpCfg<D, QT>;
+  constexpr int kProducerWarp = 4 * QT;
+  constexpr int kMmaWarp = 4 * QT + 1;
+  constexpr uint32_t kTmemCols = 256 * QT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                    // kQTiles tiles
-  uint8_t* sK = sQ + kQTiles * C::TILE_BYTES;            // STAGES tiles
+  uint8_t* sQ = smem;                                    // QT tiles
+  uint8_t* sK = sQ + QT * C::TILE_BYTES;                 // STAGES tiles
   uint8_t* sV = sK + C::STAGES * C::TILE_BYTES;          // STAGES tiles
   PpBars* bars = reinterpret_cast<PpBars*>(sV + C::STAGES * C::TILE_BYTES);
   volatile int* abort_flag = &bars->abort;
@@ -160,8 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
   int g = 0;               // query group (ring), and the CTA's first query row
   if constexpr (RING)
     while (g + 1 < p.n_qgroups && static_cast<int>(blockIdx.x) >= p.q_pair_prefix[g + 1]) ++g;
-  const int row0 = RING ? p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_pair_prefix[g]) * (kQTiles * kRows)
-                        : static_cast<int>(blockIdx.x) * (kQTiles * kRows);
+  const int row0 = RING ? p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_pair_prefix[g]) * (QT * kRows)
+                        : static_cast<int>(blockIdx.x) * (QT * kRows);
   const int q_end = RING ? min(p.q_start[g + 1], T) : T;  // rows beyond are computed but not stored
   const int ntiles = [&]() {
     if constexpr (RING) {
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int t = 0; t < kQTiles; ++t) {
+    for (int t = 0; t < QT; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 128);
       mbar_init(&bars->o_full[t], 1);
@@ -208,8 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, kQTiles * C::TILE_BYTES);
-      for (int t = 0; t < kQTiles; ++t)
+      mbar_arrive_expect_tx(&bars->q_full, QT * C::TILE_BYTES);
+      for (int t = 0; t < QT; ++t)
         for (int a = 0; a < C::NATOM; ++a)
           tma_load_4d(&p.tm_q, &bars->q_full, sQ + t * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hm,
                       row0 + t * kRows, b);
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
                 make_smem_desc(q_addr + t * C::TILE_BYTES + a * C::BLOCK_BYTES + ks * 32, 16, C::SBO, C::LAYOUT);
             const uint64_t bdesc =
                 make_smem_desc(k_addr + st * C::TILE_BYTES + a * C::BLOCK_BYTES + ks * 32, 16, C::SBO, C::LAYOUT);
-            umma_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, (a > 0 || ks > 0) ? 1u : 0u);
+            umma_ss(tmem + col_s<QT>(t), adesc, bdesc, idesc_qk, (a > 0 || ks > 0) ? 1u : 0u);
           }
         umma_commit(&bars->s_full[t]);
 #ifdef USP_TRACE
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           const uint64_t bdesc =
               make_smem_desc(v_addr + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
-          umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + col_o<QT>(t), tmem + col_s<QT>(t) + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         return true;
       };
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
       if (ok) ok = wait_k(0);
       if (ok) {
         issue_s(0, 0);
-        issue_s(1, 0);
+        if constexpr (QT == 2) issue_s(1, 0);
         umma_commit(&bars->k_empty[0]);
       }
       for (int j = 1; ok && j < ntiles; ++j) {
@@ -332,23 +337,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
         if (!(ok = wait_k(j))) break;
         const int ks = j % C::STAGES;
         issue_s(0, ks);  // after P_A(j-1) V: S_A(j) overwrites P_A(j-1)
-        if (!(ok = issue_pv(1, j - 1, vs))) break;
-        umma_commit(&bars->v_empty[vs]);
-        issue_s(1, ks);
+        if constexpr (QT == 2) {
+          if (!(ok = issue_pv(1, j - 1, vs))) break;
+          umma_commit(&bars->v_empty[vs]);
+          issue_s(1, ks);
+        } else {
+          umma_commit(&bars->v_empty[vs]);
+        }
         umma_commit(&bars->k_empty[ks]);
       }
       if (ok) {
         const int j = ntiles - 1, vs = j % C::STAGES;
         ok = wait_v(j);
         if (ok) ok = issue_pv(0, j, vs);
-        if (ok) {
-          umma_commit(&bars->o_full[0]);
-          ok = issue_pv(1, j, vs);
+        if (ok) umma_commit(&bars->o_full[0]);
+        if constexpr (QT == 2) {
+          if (ok) ok = issue_pv(1, j, vs);
+          if (ok) umma_commit(&bars->o_full[1]);
         }
-        if (ok) {
-          umma_commit(&bars->v_empty[vs]);
-          umma_commit(&bars->o_full[1]);
-        }
+        if (ok) umma_commit(&bars->v_empty[vs]);
       }
       // All MMAs this thread issued must finish before TMEM is released.
       umma_commit(&bars->drain);
@@ -360,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;             // TMEM lane = query row in the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t sc = lane_addr + col_s(t);
-    const uint32_t oc = lane_addr + col_o(t);
+    const uint32_t sc = lane_addr + col_s<QT>(t);
+    const uint32_t oc = lane_addr + col_o<QT>(t);
     const float sl2 = p.scale_log2;
     int kb_blk = 0, kb_left = 0;
     if constexpr (RING) {
@@ -530,13 +537,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pp_kernel(const __grid_const
   }
 }
 
-template <int D, bool BF16>
+template <int D, int QT, bool BF16>
 int launch_pp_d(const AttnLaunch& L, cudaStream_t stream) {
-  using C = PpCfg<D>;
-  static_assert(C::SMEM_BYTES <= 232448, "shared memory above the 227 KB per-CTA limit");
-  for (auto* fn : {attn_pp_kernel<D, BF16, false>, attn_pp_kernel<D, BF16, true>})
+  using C = PpCfg<D, QT>;
+  static_assert(C::SMEM_BYTES <= C::BUDGET, "shared memory above the per-CTA budget");
+  // Two CTAs per SM need the largest shared-memory carveout.
+  for (auto* fn : {attn_pp_kernel<D, QT, BF16, false>, attn_pp_kernel<D, QT, BF16, true>})
     if (int rc = ensure_smem_limit(reinterpret_cast<const void*>(fn), C::SMEM_BYTES,
-                                   "cudaFuncSetAttribute(attention smem)"))
+                                   "cudaFuncSetAttribute(attention smem)", QT == 1 ? 100 : -1))
       return rc;
   thread_local PpParams p;
   memset(&p, 0, sizeof(p));
@@ -548,7 +556,7 @@ int launch_pp_d(const AttnLaunch& L, cudaStream_t stream) {
   if ((rc = make_map(&p.tm_q, L.in.q, L.in.qv, L, L.tokens, C::ATOM, kRows)) != USP_OK) return rc;
   if ((rc = make_map(&p.tm_k, L.in.k, L.in.kvv, L, kv_tokens, C::ATOM, kKeys)) != USP_OK) return rc;
   if ((rc = make_map(&p.tm_v, L.in.v, L.in.kvv, L, kv_tokens, C::ATOM, kKeys)) != USP_OK) return rc;
-  if (!fill_blocks(L, kv_tokens, kQTiles * kRows, p.n_qgroups, p.n_kvblocks, p.q_start, p.q_pair_prefix, p.kv_start))
+  if (!fill_blocks(L, kv_tokens, QT * kRows, p.n_qgroups, p.n_kvblocks, p.q_start, p.q_pair_prefix, p.kv_start))
     return set_error(USP_ERR_INVALID_ARG, "internal: bad query-group or key-block table");
   p.kv_tokens = kv_tokens;
   p.lse = L.lse;
@@ -564,29 +572,38 @@ int launch_pp_d(const AttnLaunch& L, cudaStream_t stream) {
   for (int i = 0; i < L.n_heads; ++i) p.heads[i] = L.heads[i];
   const dim3 grid(p.q_pair_prefix[p.n_qgroups], L.batch * L.n_heads);
   if (ring)
-    attn_pp_kernel<D, BF16, true><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+    attn_pp_kernel<D, QT, BF16, true><<<grid, pp_threads(QT), C::SMEM_BYTES, stream>>>(p);
   else
-    attn_pp_kernel<D, BF16, false><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+    attn_pp_kernel<D, QT, BF16, false><<<grid, pp_threads(QT), C::SMEM_BYTES, stream>>>(p);
   count_launch();
-  return cuda_check(cudaGetLastError(), "attention (tcgen05, two query tiles) launch");
+  return cuda_check(cudaGetLastError(), "attention (tcgen05, 128-key tiles) launch");
 }
 
 template <bool BF16>
 int launch_pp_dtype(const AttnLaunch& L, cudaStream_t stream) {
+  if (L.kernel == USP_ATTN_TWO_CTA) {
+    switch (L.head_dim) {
+      case 64: return launch_pp_d<64, 1, BF16>(L, stream);
+      case 80: return launch_pp_d<80, 1, BF16>(L, stream);
+      default: return set_error(USP_ERR_UNSUPPORTED, "two-CTA attention: head_dim %d not built", L.head_dim);
+    }
+  }
   switch (L.head_dim) {
-    case 64: return launch_pp_d<64, BF16>(L, stream);
-    case 80: return launch_pp_d<80, BF16>(L, stream);
-    case 96: return launch_pp_d<96, BF16>(L, stream);
-    case 112: return launch_pp_d<112, BF16>(L, stream);
-    case 128: return launch_pp_d<128, BF16>(L, stream);
+    case 64: return launch_pp_d<64, 2, BF16>(L, stream);
+    case 80: return launch_pp_d<80, 2, BF16>(L, stream);
+    case 96: return launch_pp_d<96, 2, BF16>(L, stream);
+    case 112: return launch_pp_d<112, 2, BF16>(L, stream);
+    case 128: return launch_pp_d<128, 2, BF16>(L, stream);
     default: return set_error(USP_ERR_UNSUPPORTED, "two-tile attention: head_dim %d not built", L.head_dim);
   }
 }
 
 }  // namespace
 
-bool attention_pp_supported(int dtype, int head_dim) {
-  return (dtype == USP_BF16 || dtype == USP_FP16) && head_dim % 16 == 0 && head_dim >= 64 && head_dim <= 128;
+bool attention_pp_supported(int dtype, int head_dim, int kernel) {
+  if (dtype != USP_BF16 && dtype != USP_FP16) return false;
+  if (kernel == USP_ATTN_TWO_CTA) return head_dim == 64 || head_dim == 80;
+  return head_dim % 16 == 0 && head_dim >= 64 && head_dim <= 128;
 }
 
 int launch_attention_pp(const AttnLaunch& L, cudaStream_t stream) {

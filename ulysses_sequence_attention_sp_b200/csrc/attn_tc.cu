@@ -1252,10 +1252,11 @@ bool attention_tc_supported(int dtype, int head_dim) {
 
 int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream) {
   if (L.n_heads == 0 || L.batch == 0 || L.tokens == 0) return USP_OK;
-  if (L.kernel == USP_ATTN_TWO_TILE) return launch_attention_pp(L, stream);
+  if (L.kernel == USP_ATTN_TWO_TILE || L.kernel == USP_ATTN_TWO_CTA) return launch_attention_pp(L, stream);
   // Automatic: long key sequences, where one CTA per query tile would be
-  // launched, take the two-query-tile kernel. Short ones (persistent CTAs) and
-  // capped launches stay here.
+  // launched, take the two-query-tile kernel. Short ones take the same kernel
+  // with one query tile per CTA and two CTAs per SM where it is built
+  // (head_dim 64 and 80), else persistent CTAs here; capped launches stay here.
   if (L.kernel == USP_ATTN_AUTO && L.max_ctas == 0 && attention_pp_supported(L.dtype, L.head_dim)) {
     const int kv_tokens = L.kv_tokens > 0 ? L.kv_tokens : L.tokens;
     int32_t nq = 0, nk = 0, q_start[USP_MAX_WORLD + 1], q_prefix[USP_MAX_WORLD + 1], kv_start[USP_MAX_WORLD + 1];
@@ -1263,6 +1264,11 @@ int launch_attention_tc(const AttnLaunch& L, cudaStream_t stream) {
       int64_t key_tiles = 0;
       for (int k = 0; k < nk; ++k) key_tiles += (kv_start[k + 1] - kv_start[k] + kBN - 1) / kBN;
       if (key_tiles > kPersistMaxTiles) return launch_attention_pp(L, stream);
+      if (attention_pp_supported(L.dtype, L.head_dim, USP_ATTN_TWO_CTA)) {
+        AttnLaunch two_cta = L;
+        two_cta.kernel = USP_ATTN_TWO_CTA;
+        return launch_attention_pp(two_cta, stream);
+      }
     }
   }
   return L.dtype == USP_BF16 ? launch_dtype<true>(L, stream) : launch_dtype<false>(L, stream);

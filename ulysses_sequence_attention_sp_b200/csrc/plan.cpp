@@ -227,7 +227,7 @@ int cuda_check(cudaError_t e, const char* what) {
   return set_error(USP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-int ensure_smem_limit(const void* func, size_t bytes, const char* what) {
+int ensure_smem_limit(const void* func, size_t bytes, const char* what, int carveout) {
   static std::mutex m;
   static std::map<std::pair<const void*, int>, size_t> limits;
   int dev = 0;
@@ -237,6 +237,10 @@ int ensure_smem_limit(const void* func, size_t bytes, const char* what) {
   if (bytes <= set) return USP_OK;
   cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e != cudaSuccess) return cuda_check(e, what);
+  if (carveout >= 0) {
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
+    if (e != cudaSuccess) return cuda_check(e, what);
+  }
   set = bytes;
   return USP_OK;
 }
@@ -1000,11 +1004,15 @@ int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas) {
 
 int usp_plan_set_attention_kernel(usp_plan* plan, int32_t kernel) {
   if (int rc = check_plan(plan)) return rc;
-  if (kernel != USP_ATTN_AUTO && kernel != USP_ATTN_ONE_TILE && kernel != USP_ATTN_TWO_TILE)
+  if (kernel != USP_ATTN_AUTO && kernel != USP_ATTN_ONE_TILE && kernel != USP_ATTN_TWO_TILE &&
+      kernel != USP_ATTN_TWO_CTA)
     return usp::set_error(USP_ERR_INVALID_ARG, "unknown attention kernel %d", kernel);
-  if (kernel == USP_ATTN_TWO_TILE && !usp::attention_pp_supported(plan->dtype, plan->head_dim))
+  if (kernel == USP_ATTN_TWO_TILE && !usp::attention_pp_supported(plan->dtype, plan->head_dim, kernel))
     return usp::set_error(USP_ERR_UNSUPPORTED, "the two-query-tile kernel takes 16-bit inputs with head_dim a "
                           "multiple of 16 in [64, 128] (got dtype %d, head_dim %d)", plan->dtype, plan->head_dim);
+  if (kernel == USP_ATTN_TWO_CTA && !usp::attention_pp_supported(plan->dtype, plan->head_dim, kernel))
+    return usp::set_error(USP_ERR_UNSUPPORTED, "the two-CTA kernel takes 16-bit inputs with head_dim 64 or 80 "
+                          "(got dtype %d, head_dim %d)", plan->dtype, plan->head_dim);
   std::lock_guard<std::recursive_mutex> guard(plan->lock);
   plan->attn_kernel = kernel;
   return USP_OK;

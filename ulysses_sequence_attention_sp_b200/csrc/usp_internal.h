@@ -125,9 +125,10 @@ int read_pack_error(uint32_t* code, bool reset);
 int sm_count();
 
 // Raises kernel `func`'s dynamic shared-memory limit to at least `bytes` on the
-// current device. The attribute is per device, so the value set is remembered
+// current device, and (carveout >= 0) sets its preferred shared-memory carveout
+// in percent. The attributes are per device, so the value set is remembered
 // per (kernel, device); thread-safe.
-int ensure_smem_limit(const void* func, size_t bytes, const char* what);
+int ensure_smem_limit(const void* func, size_t bytes, const char* what, int carveout = -1);
 
 // The plan's device-free part (sizes, splits, grouped-query check): plan.cpp.
 int plan_geometry(usp_plan* p, int64_t batch, int64_t seq_len, int32_t heads, int32_t heads_kv, int32_t head_dim,
@@ -288,7 +289,7 @@ int make_map(CUtensorMap* map, const void* base, const AttnView& view, const Att
 
 bool attention_tc_supported(int dtype, int head_dim);
 // Two query tiles per CTA (attn_pp.cu): 16-bit, head_dim 64..128 in steps of 16.
-bool attention_pp_supported(int dtype, int head_dim);
+bool attention_pp_supported(int dtype, int head_dim, int kernel = USP_ATTN_TWO_TILE);
 int launch_attention_pp(const AttnLaunch& L, cudaStream_t stream);
 int read_pp_error(uint32_t* code, bool reset);
 int read_pp_bounds(uint32_t* code, bool reset);

@@ -290,9 +290,9 @@ class Plan:
         self.attention_ctas = int(max_ctas)
 
     def set_attention_kernel(self, kernel: str) -> None:
-        """'auto' (default), 'one_tile' or 'two_tile': which tensor-core
-        attention kernel runs (same function; see include/usp.h)."""
-        codes = {"auto": 0, "one_tile": 1, "two_tile": 2}
+        """'auto' (default), 'one_tile', 'two_tile' or 'two_cta': which
+        tensor-core attention kernel runs (same function; see include/usp.h)."""
+        codes = {"auto": 0, "one_tile": 1, "two_tile": 2, "two_cta": 3}
         if kernel not in codes:
             raise UspError(USP_ERR_INVALID_ARG, f"attention kernel must be one of {sorted(codes)}")
         _check(_lib.usp_plan_set_attention_kernel(self.handle, codes[kernel]))
