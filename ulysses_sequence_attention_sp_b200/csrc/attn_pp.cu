@@ -30,6 +30,7 @@
 // stale maximum is kept otherwise: exact, since numerator and denominator use
 // the same maximum). A tile's O is only ever written by its own P.V, which
 // has completed whenever the tile's next S has (one commit covers both).
+#include <algorithm>
 #include <cmath>
 
 #include "device_common.cuh"
@@ -42,13 +43,15 @@ __device__ uint32_t g_pp_error;   // first wait that ran out (site code), 0 if n
 __device__ uint32_t g_pp_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
 
 // Pipeline trace (built only with -DUSP_TRACE): clock64() at pipeline events
-// of CTA 7, [event][key tile]; read with usp_debug_read_trace_pp.
+// of one CTA (query tile group min(7, half the groups), batch-head min(3, last)),
+// [event][key tile]; read with usp_debug_read_trace_pp.
 #ifdef USP_TRACE
 constexpr int kPpTraceEvents = 16, kPpTraceTiles = 256;
 __device__ unsigned long long g_pp_trace[kPpTraceEvents][kPpTraceTiles];
 #define PP_TRACE(ev, j)                                                                   \
   do {                                                                                    \
-    if (blockIdx.x == 7 && blockIdx.y == 0 && (j) < kPpTraceTiles) g_pp_trace[(ev)][(j)] = clock64(); \
+    if (blockIdx.x == min(7u, gridDim.x / 2) && blockIdx.y == min(3u, gridDim.y - 1) && (j) < kPpTraceTiles) \
+      g_pp_trace[(ev)][(j)] = clock64();                                                  \
   } while (0)
 #else
 #define PP_TRACE(ev, j) \
@@ -92,10 +95,11 @@ struct PpCfg {
 };
 
 struct PpBars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;  // Q tiles landed; the last S of the item that read them done
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t v_full[kMaxStages], v_empty[kMaxStages];
   uint64_t s_full[kMaxQTiles], p_full[kMaxQTiles], o_full[kMaxQTiles];
+  uint64_t o_free[kMaxQTiles];  // the epilogue has read O (one arrival per softmax warp)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -111,8 +115,9 @@ struct PpParams {
   int32_t kv_group, q_head_base, kv_head_base;  // k/v head of query head h: (q_head_base + h) / kv_group - kv_head_base
   float scale_log2;
   int32_t n_qgroups, n_kvblocks;
+  int32_t n_items;                           // (query-tile group, batch, head) items of the launch
   int32_t q_start[USP_MAX_WORLD + 1];
-  int32_t q_pair_prefix[USP_MAX_WORLD + 1];  // CTAs (query-tile pairs) before group g
+  int32_t q_pair_prefix[USP_MAX_WORLD + 1];  // query-tile groups before query group g
   int32_t kv_start[USP_MAX_WORLD + 1];
   uint16_t heads[USP_MAX_HEADS];
 };
@@ -137,6 +142,28 @@ __device__ __forceinline__ KeyTile key_tile(const PpParams& p, int g, int j) {
   return KeyTile{0, 0};  // not reached for j < the group's tile count
 }
 
+// Work item `it` of a launch: query-tile group x (QT tiles of 128 rows) of one
+// (batch, head), x fastest, so that CTAs running at the same time share K and V.
+struct PpItem {
+  int b, hm, hk, g, row0, q_end;
+};
+__device__ __forceinline__ PpItem pp_item(const PpParams& p, int it, int qt, bool ring) {
+  const int nx = p.q_pair_prefix[p.n_qgroups];
+  const int bh = it / nx;
+  const int x = it - bh * nx;
+  const int hi = bh / p.batch;
+  PpItem w;
+  w.b = bh - hi * p.batch;
+  w.hm = p.heads[hi];
+  w.hk = (p.q_head_base + w.hm) / p.kv_group - p.kv_head_base;  // grouped-query attention
+  w.g = 0;                                                       // query group (ring)
+  if (ring)
+    while (w.g + 1 < p.n_qgroups && x >= p.q_pair_prefix[w.g + 1]) ++w.g;
+  w.row0 = ring ? p.q_start[w.g] + (x - p.q_pair_prefix[w.g]) * (qt * kRows) : x * (qt * kRows);
+  w.q_end = ring ? min(p.q_start[w.g + 1], p.tokens) : p.tokens;  // rows beyond are computed but not stored
+  return w;
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return bf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
@@ -157,17 +184,10 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int hi = blockIdx.y / p.batch;
-  const int b = blockIdx.y - hi * p.batch;
-  const int hm = p.heads[hi];
-  const int hk = (p.q_head_base + hm) / p.kv_group - p.kv_head_base;  // grouped-query attention
   const int T = p.tokens;  // query rows; the plain kernel also takes them as keys
-  int g = 0;               // query group (ring), and the CTA's first query row
-  if constexpr (RING)
-    while (g + 1 < p.n_qgroups && static_cast<int>(blockIdx.x) >= p.q_pair_prefix[g + 1]) ++g;
-  const int row0 = RING ? p.q_start[g] + (static_cast<int>(blockIdx.x) - p.q_pair_prefix[g]) * (QT * kRows)
-                        : static_cast<int>(blockIdx.x) * (QT * kRows);
-  const int q_end = RING ? min(p.q_start[g + 1], T) : T;  // rows beyond are computed but not stored
+  // Key tiles per item (every item walks all keys). A CTA takes items
+  // blockIdx.x, blockIdx.x + gridDim.x, ...; tile j of its k-th item is its
+  // (k * ntiles + j)-th, which fixes every ring stage and barrier phase.
   const int ntiles = [&]() {
     if constexpr (RING) {
       int n = 0;
@@ -176,9 +196,15 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
     }
     return (T + kKeys - 1) / kKeys;
   }();
+  // Two-tile CTAs take exactly one item (k = 0 below, known to the compiler).
+  const int it0 = blockIdx.x, it_step = gridDim.x;
+  const int it_end = QT == 2 ? min(it0 + 1, p.n_items) : p.n_items;
 
+  // One-tile CTAs trace their start-up and epilogues in the second tile's slots.
+  if (QT == 1 && threadIdx.x == 0) PP_TRACE(9, 0);
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
@@ -189,6 +215,7 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 128);
       mbar_init(&bars->o_full[t], 1);
+      mbar_init(&bars->o_free[t], 4);
     }
     mbar_init(&bars->drain, 1);
     // An earlier launch or CTA recorded an error: this CTA does no work.
@@ -204,6 +231,7 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const bool skip = bars->abort != 0;  // uniform: read after the barrier, before any wait
+  if (QT == 1 && threadIdx.x == 0) PP_TRACE(10, 0);
 
   if (skip) {
     // fall through to the common exit
@@ -213,50 +241,45 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
       prefetch_tensormap(&p.tm_q);
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, QT * C::TILE_BYTES);
-      for (int t = 0; t < QT; ++t)
-        for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_q, &bars->q_full, sQ + t * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hm,
-                      row0 + t * kRows, b);
-      auto key0_of = [&](int j) { return RING ? key_tile(p, g, j).key0 : j * kKeys; };
-      // K of tile j into stage j % STAGES once the S products of tile j - STAGES are done.
-      auto load_k = [&](int j) -> bool {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES &&
-            !mbar_wait(&bars->k_empty[st], ((j / C::STAGES) - 1) & 1, abort_flag, &g_pp_error, 40, kWaitLimitNs))
+      int nk = 0, nv = 0, nq = 0;  // K tiles, V tiles and Q groups issued, over all items
+      // K (or V) of tile j of item w: the n-th tile of the CTA goes to stage
+      // n % STAGES once the products that read tile n - STAGES are done.
+      auto load_kv = [&](bool v, const PpItem& w, int j) -> bool {
+        int& n = v ? nv : nk;
+        const int st = n % C::STAGES;
+        uint64_t* full = v ? &bars->v_full[st] : &bars->k_full[st];
+        uint64_t* empty = v ? &bars->v_empty[st] : &bars->k_empty[st];
+        if (n >= C::STAGES &&
+            !mbar_wait(empty, ((n / C::STAGES) - 1) & 1, abort_flag, &g_pp_error, 40 + v, kWaitLimitNs))
           return false;
-        mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
-        const int key0 = key0_of(j);
+        mbar_arrive_expect_tx(full, C::TILE_BYTES);
+        const int key0 = RING ? key_tile(p, w.g, j).key0 : j * kKeys;
+        uint8_t* dst = (v ? sV : sK) + st * C::TILE_BYTES;
         for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_k, &bars->k_full[st], sK + st * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hk,
-                      key0, b);
+          tma_load_4d(v ? &p.tm_v : &p.tm_k, full, dst + a * C::BLOCK_BYTES, a * C::ATOM, w.hk, key0, w.b);
+        ++n;
         return true;
       };
-      // V of tile j once the P V products of tile j - STAGES are done.
-      auto load_v = [&](int j) -> bool {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES &&
-            !mbar_wait(&bars->v_empty[st], ((j / C::STAGES) - 1) & 1, abort_flag, &g_pp_error, 41, kWaitLimitNs))
-          return false;
-        mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
-        const int key0 = key0_of(j);
-        for (int a = 0; a < C::NATOM; ++a)
-          tma_load_4d(&p.tm_v, &bars->v_full[st], sV + st * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, hk,
-                      key0, b);
-        return true;
-      };
-      // Issue order follows consumption: K(0), then K(j+1) before V(j).
-      int nk = 0, nv = 0;
-      bool go = load_k(0);
-      nk += go;
-      for (int j = 0; go && j < ntiles; ++j) {
-        if (j + 1 < ntiles) {
-          go = load_k(j + 1);
-          nk += go;
-        }
+      bool go = true;
+      for (int it = it0, k = 0; go && it < it_end; it += it_step, ++k) {
+        if constexpr (QT == 2) k = 0;
+        const PpItem w = pp_item(p, it, QT, RING);
+        go = load_kv(false, w, 0);
+        // Q of this item once the last S of the previous one (which read Q) is done.
+        if (go && k > 0)
+          go = mbar_wait(&bars->q_empty, (k - 1) & 1, abort_flag, &g_pp_error, 39, kWaitLimitNs);
         if (go) {
-          go = load_v(j);
-          nv += go;
+          mbar_arrive_expect_tx(&bars->q_full, QT * C::TILE_BYTES);
+          for (int t = 0; t < QT; ++t)
+            for (int a = 0; a < C::NATOM; ++a)
+              tma_load_4d(&p.tm_q, &bars->q_full, sQ + t * C::TILE_BYTES + a * C::BLOCK_BYTES, a * C::ATOM, w.hm,
+                          w.row0 + t * kRows, w.b);
+          ++nq;
+        }
+        // Issue order follows consumption: K(0), then K(j+1) before V(j).
+        for (int j = 0; go && j < ntiles; ++j) {
+          if (j + 1 < ntiles) go = load_kv(false, w, j + 1);
+          if (go) go = load_kv(true, w, j);
         }
       }
       if (*abort_flag) {
@@ -265,7 +288,7 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
           mbar_wait_drain(&bars->k_full[j % C::STAGES], (j / C::STAGES) & 1, kDrainLimitNs);
         for (int j = (nv > C::STAGES ? nv - C::STAGES : 0); j < nv; ++j)
           mbar_wait_drain(&bars->v_full[j % C::STAGES], (j / C::STAGES) & 1, kDrainLimitNs);
-        mbar_wait_drain(&bars->q_full, 0, kDrainLimitNs);
+        if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1, kDrainLimitNs);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -276,13 +299,9 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, &g_pp_error, 42, kWaitLimitNs);
-      tc_fence_after();
       // S_t = Q_t K^T for the K tile in ring stage st (already landed).
-#ifdef USP_TRACE
-      int s_count[2] = {0, 0};
-#endif
-      auto issue_s = [&](int t, int st) {
+      auto issue_s = [&](int t, int st, int jg) {
+        PP_TRACE(t, jg);
 #pragma unroll
         for (int a = 0; a < C::NATOM; ++a)
 #pragma unroll
@@ -294,15 +313,17 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
             umma_ss(tmem + col_s<QT>(t), adesc, bdesc, idesc_qk, (a > 0 || ks > 0) ? 1u : 0u);
           }
         umma_commit(&bars->s_full[t]);
-#ifdef USP_TRACE
-        const int si = s_count[t]++;
-        PP_TRACE(t, si);
-#endif
+        if (QT == 1) PP_TRACE(15, jg);
       };
-      // O_t += P_t(j) V_j once the softmax of tile t has stored P_t(j) (V stage st landed).
-      auto issue_pv = [&](int t, int j, int st) -> bool {
-        if (!mbar_wait(&bars->p_full[t], j & 1, abort_flag, &g_pp_error, 43 + t, kWaitLimitNs)) return false;
-        PP_TRACE(2 + t, j);
+      // O_t += P_t V for the CTA's tile jg (tile j of its item) once the softmax
+      // of tile t has stored P_t; before an item's first P V, the epilogue of
+      // the CTA's previous item (k - 1) must have read O_t.
+      auto issue_pv = [&](int t, int j, int jg, int k, int st) -> bool {
+        if (j == 0 && k > 0 &&
+            !mbar_wait(&bars->o_free[t], (k - 1) & 1, abort_flag, &g_pp_error, 56 + t, kWaitLimitNs))
+          return false;
+        if (!mbar_wait(&bars->p_full[t], jg & 1, abort_flag, &g_pp_error, 43 + t, kWaitLimitNs)) return false;
+        PP_TRACE(2 + t, jg);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
@@ -312,47 +333,56 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
         }
         return true;
       };
-      auto wait_k = [&](int j) {
-        const int st = j % C::STAGES;
-        const bool r = mbar_wait(&bars->k_full[st], (j / C::STAGES) & 1, abort_flag, &g_pp_error, 45, kWaitLimitNs);
+      auto wait_k = [&](int jg) {
+        const int st = jg % C::STAGES;
+        const bool r = mbar_wait(&bars->k_full[st], (jg / C::STAGES) & 1, abort_flag, &g_pp_error, 45, kWaitLimitNs);
         tc_fence_after();
         return r;
       };
-      auto wait_v = [&](int j) {
-        const int st = j % C::STAGES;
-        const bool r = mbar_wait(&bars->v_full[st], (j / C::STAGES) & 1, abort_flag, &g_pp_error, 46, kWaitLimitNs);
+      auto wait_v = [&](int jg) {
+        const int st = jg % C::STAGES;
+        const bool r = mbar_wait(&bars->v_full[st], (jg / C::STAGES) & 1, abort_flag, &g_pp_error, 46, kWaitLimitNs);
         tc_fence_after();
         return r;
       };
-      if (ok) ok = wait_k(0);
-      if (ok) {
-        issue_s(0, 0);
-        if constexpr (QT == 2) issue_s(1, 0);
-        umma_commit(&bars->k_empty[0]);
-      }
-      for (int j = 1; ok && j < ntiles; ++j) {
-        const int vs = (j - 1) % C::STAGES;
-        if (!(ok = wait_v(j - 1))) break;
-        if (!(ok = issue_pv(0, j - 1, vs))) break;
-        if (!(ok = wait_k(j))) break;
-        const int ks = j % C::STAGES;
-        issue_s(0, ks);  // after P_A(j-1) V: S_A(j) overwrites P_A(j-1)
-        if constexpr (QT == 2) {
-          if (!(ok = issue_pv(1, j - 1, vs))) break;
-          umma_commit(&bars->v_empty[vs]);
-          issue_s(1, ks);
-        } else {
-          umma_commit(&bars->v_empty[vs]);
+      bool ok = true;
+      for (int it = it0, k = 0; ok && it < it_end; it += it_step, ++k) {
+        if constexpr (QT == 2) k = 0;
+        const int base = k * ntiles;  // the CTA's tile index of this item's tile 0
+        ok = mbar_wait(&bars->q_full, k & 1, abort_flag, &g_pp_error, 42, kWaitLimitNs);
+        tc_fence_after();
+        if (QT == 1) PP_TRACE(11, k);
+        if (ok) ok = wait_k(base);
+        if (QT == 1) PP_TRACE(14, k);
+        if (!ok) break;
+        // S_t(0) overwrites P_t of the previous item, whose P V was issued before.
+        issue_s(0, base % C::STAGES, base);
+        if constexpr (QT == 2) issue_s(1, base % C::STAGES, base);
+        umma_commit(&bars->k_empty[base % C::STAGES]);
+        for (int j = 1; ok && j < ntiles; ++j) {
+          const int vs = (base + j - 1) % C::STAGES;
+          if (!(ok = wait_v(base + j - 1))) break;
+          if (!(ok = issue_pv(0, j - 1, base + j - 1, k, vs))) break;
+          if (!(ok = wait_k(base + j))) break;
+          const int ks = (base + j) % C::STAGES;
+          issue_s(0, ks, base + j);  // after P_A(j-1) V: S_A(j) overwrites P_A(j-1)
+          if constexpr (QT == 2) {
+            if (!(ok = issue_pv(1, j - 1, base + j - 1, k, vs))) break;
+            umma_commit(&bars->v_empty[vs]);
+            issue_s(1, ks, base + j);
+          } else {
+            umma_commit(&bars->v_empty[vs]);
+          }
+          umma_commit(&bars->k_empty[ks]);
         }
-        umma_commit(&bars->k_empty[ks]);
-      }
-      if (ok) {
-        const int j = ntiles - 1, vs = j % C::STAGES;
-        ok = wait_v(j);
-        if (ok) ok = issue_pv(0, j, vs);
+        if (!ok) break;
+        umma_commit(&bars->q_empty);  // every S of this item issued: Q may be replaced once they are done
+        const int j = ntiles - 1, jg = base + j, vs = jg % C::STAGES;
+        ok = wait_v(jg);
+        if (ok) ok = issue_pv(0, j, jg, k, vs);
         if (ok) umma_commit(&bars->o_full[0]);
         if constexpr (QT == 2) {
-          if (ok) ok = issue_pv(1, j, vs);
+          if (ok) ok = issue_pv(1, j, jg, k, vs);
           if (ok) umma_commit(&bars->o_full[1]);
         }
         if (ok) umma_commit(&bars->v_empty[vs]);
@@ -370,118 +400,135 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
     const uint32_t sc = lane_addr + col_s<QT>(t);
     const uint32_t oc = lane_addr + col_o<QT>(t);
     const float sl2 = p.scale_log2;
-    int kb_blk = 0, kb_left = 0;
-    if constexpr (RING) {
-      kb_blk = g % p.n_kvblocks;
-      kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
-    }
-    float m = -INFINITY;  // running maximum, log2 domain
-    float l = 0.f;        // running denominator
+    const bool tr0 = quarter == 0 && lane == 0;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, abort_flag, &g_pp_error, 50 + t,
+    for (int it = it0, k = 0; ok && it < it_end; it += it_step, ++k) {
+      if constexpr (QT == 2) k = 0;
+      int kb_blk = 0, kb_left = 0;
+      if constexpr (RING) {
+        kb_blk = pp_item(p, it, QT, RING).g % p.n_kvblocks;
+        kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+      }
+      float m = -INFINITY;  // running maximum, log2 domain
+      float l = 0.f;        // running denominator
+      for (int j = 0; j < ntiles; ++j) {
+        const int jg = k * ntiles + j;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], jg & 1, abort_flag, &g_pp_error, 50 + t,
+                                               kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        if (tr0) PP_TRACE(4 + 5 * t, jg);
+        tc_fence_after();
+        uint32_t sr[kKeys];
+#pragma unroll
+        for (int c = 0; c < kKeys; c += 32) tmem_ld32(sc + c, sr + c);
+        tmem_wait_ld();
+        if (tr0) PP_TRACE(5 + 5 * t, jg);
+        float* s = reinterpret_cast<float*>(sr);
+        const int valid = RING ? kb_left : T - j * kKeys;  // valid keys of this tile (>= kKeys: all)
+        if (valid < kKeys) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        // Row maximum: eight independent three-input chains, then a tree.
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float a = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+          for (int c = i + 16; c < kKeys; c += 16) a = max3(a, s[c], s[c + 8]);
+          mx8[i] = a;
+        }
+        const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_new = fmaxf(m, mx * sl2);
+        if (tr0) PP_TRACE(6 + 5 * t, jg);
+        if (j == 0) {
+          m = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
+          // O holds sum_{i<j} exp2(s_i - m) v_i (its last P V completed before
+          // this tile's S did); bring it to the new maximum.
+          const float alpha = ex2_approx(m - m_new);
+          m = m_new;
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(oc + c * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(oc + c * 16, o);
+          }
+          tmem_wait_st();
+        }
+        // p = 2^(s*scale*log2e - m), packed to the input type, written over the
+        // first 64 columns of S (already in registers) in two halves. Masked
+        // entries (s = -inf) give exactly 0.
+        // The scaling and the row sum run on packed fp32 pairs (one instruction
+        // per two values). Measured and not kept: rounding P on the integer pipe
+        // instead of cvt (10% slower); a quarter or half of the exponentials as a
+        // degree-3 polynomial on the FMA pipe (4-5% slower).
+        const uint64_t scale2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(-m, -m);
+        uint64_t acc2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[64 * h + c], s[64 * h + c + 1]), scale2, negm2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            acc2[(c >> 1) & 3] = f2_add(acc2[(c >> 1) & 3], f2_pack(p0, p1));
+            pk[c / 2] = pack2(p0, p1, BF16);
+          }
+          tmem_st32(sc + 32 * h, pk);
+        }
+        float a0, a1, a2, a3, a4, a5, a6, a7;
+        f2_unpack(acc2[0], a0, a1);
+        f2_unpack(acc2[1], a2, a3);
+        f2_unpack(acc2[2], a4, a5);
+        f2_unpack(acc2[3], a6, a7);
+        l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+        if (tr0) PP_TRACE(7 + 5 * t, jg);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[t]);
+        if (tr0) PP_TRACE(8 + 5 * t, jg);
+        if constexpr (RING) {
+          kb_left -= kKeys;
+          if (kb_left <= 0) {
+            kb_blk = kb_blk == 0 ? p.n_kvblocks - 1 : kb_blk - 1;
+            kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
+          }
+        }
+      }
+      if (!ok) break;
+      // Epilogue: O of this tile, normalised, to the rows' destinations.
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], k & 1, abort_flag, &g_pp_error, 52 + t,
                                              kWaitLimitNs))) {
         ok = false;
         break;
       }
-      const bool tr0 = (warp & 3) == 0 && lane == 0;
-      if (tr0) PP_TRACE(4 + 5 * t, j);
       tc_fence_after();
-      uint32_t sr[kKeys];
+      if (QT == 1 && tr0) PP_TRACE(12, k);
+      // The whole row of O in one round of TMEM loads; then O may be overwritten.
+      uint32_t o[D];
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 32) tmem_ld32(sc + c, sr + c);
+      for (int c = 0; c < D / 16; ++c) tmem_ld16(oc + c * 16, *reinterpret_cast<uint32_t(*)[16]>(o + c * 16));
       tmem_wait_ld();
-      if (tr0) PP_TRACE(5 + 5 * t, j);
-      float* s = reinterpret_cast<float*>(sr);
-      const int valid = RING ? kb_left : T - j * kKeys;  // valid keys of this tile (>= kKeys: all)
-      if (valid < kKeys) {
-#pragma unroll
-        for (int c = 0; c < kKeys; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      // Row maximum: eight independent three-input chains, then a tree.
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float a = fmaxf(s[i], s[i + 8]);
-#pragma unroll
-        for (int c = i + 16; c < kKeys; c += 16) a = max3(a, s[c], s[c + 8]);
-        mx8[i] = a;
-      }
-      const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-      const float m_new = fmaxf(m, mx * sl2);
-      if (tr0) PP_TRACE(6 + 5 * t, j);
-      if (j == 0) {
-        m = m_new;
-      } else if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
-        // O holds sum_{i<j} exp2(s_i - m) v_i (its last P V completed before
-        // this tile's S did); bring it to the new maximum.
-        const float alpha = ex2_approx(m - m_new);
-        m = m_new;
-        l *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(oc + c * 16, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(oc + c * 16, o);
-        }
-        tmem_wait_st();
-      }
-      // p = 2^(s*scale*log2e - m), packed to the input type, written over the
-      // first 64 columns of S (already in registers) in two halves. Masked
-      // entries (s = -inf) give exactly 0.
-      // The scaling and the row sum run on packed fp32 pairs (one instruction
-      // per two values). Measured and not kept: rounding P on the integer pipe
-      // instead of cvt (10% slower); a quarter or half of the exponentials as a
-      // degree-3 polynomial on the FMA pipe (4-5% slower).
-      const uint64_t scale2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-m, -m);
-      uint64_t acc2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[64 * h + c], s[64 * h + c + 1]), scale2, negm2), x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          acc2[(c >> 1) & 3] = f2_add(acc2[(c >> 1) & 3], f2_pack(p0, p1));
-          pk[c / 2] = pack2(p0, p1, BF16);
-        }
-        tmem_st32(sc + 32 * h, pk);
-      }
-      float a0, a1, a2, a3, a4, a5, a6, a7;
-      f2_unpack(acc2[0], a0, a1);
-      f2_unpack(acc2[1], a2, a3);
-      f2_unpack(acc2[2], a4, a5);
-      f2_unpack(acc2[3], a6, a7);
-      l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-      if (tr0) PP_TRACE(7 + 5 * t, j);
-      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[t]);
-      if (tr0) PP_TRACE(8 + 5 * t, j);
-      if constexpr (RING) {
-        kb_left -= kKeys;
-        if (kb_left <= 0) {
-          kb_blk = kb_blk == 0 ? p.n_kvblocks - 1 : kb_blk - 1;
-          kb_left = p.kv_start[kb_blk + 1] - p.kv_start[kb_blk];
-        }
-      }
-    }
-    // Epilogue: O of this tile, normalised, to the rows' destinations.
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], 0, abort_flag, &g_pp_error, 52 + t,
-                                                 kWaitLimitNs))) {
-      tc_fence_after();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_free[t]);
       const float inv_l = 1.f / l;
-      const int tr = row0 + t * kRows + row;  // row of the full sequence
-      const bool row_ok = tr < q_end;
+      const PpItem w = pp_item(p, it, QT, RING);
+      const int tr = w.row0 + t * kRows + row;  // row of the full sequence
+      const bool row_ok = tr < w.q_end;
       if (p.lse != nullptr && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
-        const int64_t li = (static_cast<int64_t>(hm) * p.batch + b) * T + tr;
+        const int64_t li = (static_cast<int64_t>(w.hm) * p.batch + w.b) * T + tr;
         if (in_bounds(li, 1, p.lse_ext, 22, &g_pp_bounds)) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
       }
       const AttnOut& out = p.out;
@@ -502,30 +549,18 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
         }
       }
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(oc + c * 16, o);
-        tmem_wait_ld();
-        uint4 w0, w1;
-        w0.x = pack2(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l, BF16);
-        w0.y = pack2(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l, BF16);
-        w0.z = pack2(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l, BF16);
-        w0.w = pack2(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l, BF16);
-        w1.x = pack2(__uint_as_float(o[8]) * inv_l, __uint_as_float(o[9]) * inv_l, BF16);
-        w1.y = pack2(__uint_as_float(o[10]) * inv_l, __uint_as_float(o[11]) * inv_l, BF16);
-        w1.z = pack2(__uint_as_float(o[12]) * inv_l, __uint_as_float(o[13]) * inv_l, BF16);
-        w1.w = pack2(__uint_as_float(o[14]) * inv_l, __uint_as_float(o[15]) * inv_l, BF16);
-        for (int sg = seg_lo; sg < seg_hi; ++sg) {
-          const int64_t rows_s = out.prefix + out.seg_len[sg];
-          const int64_t elem =
-              ((static_cast<int64_t>(b) * rows_s + row_in_seg) * out.out_heads + hm - out.head_base) * D + c * 16;
-          if (!in_bounds(elem, 16, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds))
-            continue;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem);
-          dst[0] = w0;
-          dst[1] = w1;
-        }
+      for (int i = 0; i < D / 2; ++i)
+        o[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, BF16);
+      for (int sg = seg_lo; sg < seg_hi; ++sg) {
+        const int64_t rows_s = out.prefix + out.seg_len[sg];
+        const int64_t elem =
+            ((static_cast<int64_t>(w.b) * rows_s + row_in_seg) * out.out_heads + w.hm - out.head_base) * D;
+        if (!in_bounds(elem, D, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds)) continue;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
       }
+      if (QT == 1 && tr0) PP_TRACE(13, k);
     }
   }
 
@@ -570,7 +605,14 @@ int launch_pp_d(const AttnLaunch& L, cudaStream_t stream) {
   p.n_heads = L.n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(L.scale) * 1.4426950408889634);
   for (int i = 0; i < L.n_heads; ++i) p.heads[i] = L.heads[i];
-  const dim3 grid(p.q_pair_prefix[p.n_qgroups], L.batch * L.n_heads);
+  const int64_t items = static_cast<int64_t>(p.q_pair_prefix[p.n_qgroups]) * L.batch * L.n_heads;
+  if (items > INT32_MAX) return set_error(USP_ERR_UNSUPPORTED, "attention: %lld query tiles in one launch", (long long)items);
+  p.n_items = static_cast<int32_t>(items);
+  // Two query tiles: one CTA per item. One query tile: two CTAs per SM walk
+  // the items, each starting an item's loads and first Q K^T under the end of
+  // the one before.
+  const int64_t ctas = QT == 2 ? items : std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
+  const dim3 grid(static_cast<unsigned>(ctas));
   if (ring)
     attn_pp_kernel<D, QT, BF16, true><<<grid, pp_threads(QT), C::SMEM_BYTES, stream>>>(p);
   else
