@@ -86,7 +86,12 @@ struct PpCfg {
   static constexpr int BLOCK_BYTES = 128 * ROWB;         // one atom-column block of a 128-row tile
   static constexpr int TILE_BYTES = 128 * D * 2;         // a Q, K or V tile: NATOM blocks
   static constexpr int KSTEPS = ATOM / 16;
-  static constexpr int FIXED = QT * TILE_BYTES + 1024 + 2048;  // Q tiles, base alignment, barriers
+  // One-tile CTAs stage each softmax warp's output rows, half a row at a time,
+  // so that its global stores run along rows (16-byte chunks; a padded stride
+  // when a half row is an even number of chunks, against bank conflicts).
+  static constexpr int STG_STRIDE = (D / 16) % 2 ? D : D + 16;
+  static constexpr int STG_BYTES = QT == 1 ? 4 * 32 * STG_STRIDE : 0;
+  static constexpr int FIXED = QT * TILE_BYTES + STG_BYTES + 1024 + 2048;  // Q, staging, base alignment, barriers
   // Shared memory per CTA: all of it (227 KB) for one CTA per SM; for two,
   // half of the SM's 228 KB less the 1 KB the hardware reserves per CTA.
   static constexpr int BUDGET = QT == 2 ? 232448 : 115712;
@@ -179,7 +184,8 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
   uint8_t* sQ = smem;                                    // QT tiles
   uint8_t* sK = sQ + QT * C::TILE_BYTES;                 // STAGES tiles
   uint8_t* sV = sK + C::STAGES * C::TILE_BYTES;          // STAGES tiles
-  PpBars* bars = reinterpret_cast<PpBars*>(sV + C::STAGES * C::TILE_BYTES);
+  uint8_t* sStg = sV + C::STAGES * C::TILE_BYTES;        // output staging (one-tile CTAs)
+  PpBars* bars = reinterpret_cast<PpBars*>(sStg + C::STG_BYTES);
   volatile int* abort_flag = &bars->abort;
 
   const int warp = threadIdx.x >> 5;
@@ -551,12 +557,48 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
 #pragma unroll
       for (int i = 0; i < D / 2; ++i)
         o[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, BF16);
-      for (int sg = seg_lo; sg < seg_hi; ++sg) {
+      // This row's destination in segment sg (null: out of range).
+      auto row_dst = [&](int sg) -> uint16_t* {
         const int64_t rows_s = out.prefix + out.seg_len[sg];
         const int64_t elem =
             ((static_cast<int64_t>(w.b) * rows_s + row_in_seg) * out.out_heads + w.hm - out.head_base) * D;
-        if (!in_bounds(elem, D, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds)) continue;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out.seg_ptr[sg]) + elem);
+        if (!in_bounds(elem, D, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds))
+          return nullptr;
+        return static_cast<uint16_t*>(out.seg_ptr[sg]) + elem;
+      };
+      int sg_direct = seg_lo;  // segments this thread writes itself, from its registers
+      if constexpr (QT == 1) {
+        // The warp's 32 rows, half a row per round, through its staging block:
+        // each thread writes its half row, then the warp stores the block in
+        // row-major order, consecutive threads writing consecutive 16-byte
+        // chunks of a row. The first segment goes this way; a replicated
+        // prefix row's other segments are written directly below.
+        constexpr int CH = D / 16;  // 16-byte chunks per half row
+        const uint64_t my_dst = row_ok ? reinterpret_cast<uint64_t>(row_dst(seg_lo)) : 0;
+        const uint32_t stg = smem_u32(sStg) + quarter * (32 * C::STG_STRIDE);
+        sg_direct = seg_lo + 1;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            const int i = h * (D / 4) + 4 * c;
+            st_shared_v4(stg + lane * C::STG_STRIDE + c * 16, o[i], o[i + 1], o[i + 2], o[i + 3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int st = 0; st < CH; ++st) {
+            const int q = st * 32 + lane;  // chunk q of the block: row q / CH, chunk q % CH
+            const int r = q / CH, c = q - r * CH;
+            const uint4 v = ld_shared_v4(stg + r * C::STG_STRIDE + c * 16);
+            const uint64_t d = __shfl_sync(0xffffffffu, my_dst, r);
+            if (d != 0) reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(d) + h * (D / 2))[c] = v;
+          }
+          __syncwarp();
+        }
+      }
+      for (int sg = sg_direct; sg < seg_hi; ++sg) {
+        uint4* dst = reinterpret_cast<uint4*>(row_dst(sg));
+        if (dst == nullptr) continue;
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
       }
