@@ -50,13 +50,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // error in the device-wide word *err; the caller then skips the rest of its
 // work and goes to the common exit. The first thread to give up records
 // `site` in *err (first writer wins) and sets *abort.
+// The barrier is polled back to back; the abort flag, the error word (a
+// global load, hundreds of cycles) and the clock are checked only every 32nd
+// poll, so that a completion is seen within one poll, not one global load.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err, uint32_t site, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (;;) {
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
-    {
+    if ((n & 31u) == 0) {
       if (*abort || *reinterpret_cast<volatile uint32_t*>(err) != 0) {
         *abort = 1;
         return false;
