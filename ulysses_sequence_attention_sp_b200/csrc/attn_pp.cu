@@ -103,7 +103,8 @@ struct PpBars {
   uint64_t q_full, q_empty;  // Q tiles landed; the last S of the item that read them done
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-  uint64_t s_full[kMaxQTiles], p_full[kMaxQTiles], o_full[kMaxQTiles];
+  uint64_t s_full[kMaxQTiles], o_full[kMaxQTiles];
+  uint64_t p_half[kMaxQTiles], p_full[kMaxQTiles];  // first 64 keys of P stored; all of P stored
   uint64_t o_free[kMaxQTiles];  // the epilogue has read O (one arrival per softmax warp)
   uint64_t drain;
   uint32_t tmem_base;
@@ -219,6 +220,7 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_half[t], 128);
       mbar_init(&bars->p_full[t], 128);
       mbar_init(&bars->o_full[t], 1);
       mbar_init(&bars->o_free[t], 4);
@@ -321,21 +323,28 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
         umma_commit(&bars->s_full[t]);
         if (QT == 1) PP_TRACE(15, jg);
       };
-      // O_t += P_t V for the CTA's tile jg (tile j of its item) once the softmax
-      // of tile t has stored P_t; before an item's first P V, the epilogue of
-      // the CTA's previous item (k - 1) must have read O_t.
+      // O_t += P_t V for the CTA's tile jg (tile j of its item): the products
+      // over the first 64 keys once the softmax of tile t has stored that half
+      // of P_t, the rest once it has stored all of it. Before an item's first
+      // P V, the epilogue of the CTA's previous item (k - 1) must have read O_t.
       auto issue_pv = [&](int t, int j, int jg, int k, int st) -> bool {
         if (j == 0 && k > 0 &&
             !mbar_wait(&bars->o_free[t], (k - 1) & 1, abort_flag, &g_pp_error, 56 + t, kWaitLimitNs))
           return false;
-        if (!mbar_wait(&bars->p_full[t], jg & 1, abort_flag, &g_pp_error, 43 + t, kWaitLimitNs)) return false;
-        PP_TRACE(2 + t, jg);
-        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t bdesc =
-              make_smem_desc(v_addr + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
-          umma_ts(tmem + col_o<QT>(t), tmem + col_s<QT>(t) + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(h == 0 ? &bars->p_half[t] : &bars->p_full[t], jg & 1, abort_flag, &g_pp_error,
+                         h == 0 ? 58 + t : 43 + t, kWaitLimitNs))
+            return false;
+          if (h == 0) PP_TRACE(2 + t, jg);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+            const uint64_t bdesc =
+                make_smem_desc(v_addr + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
+            umma_ts(tmem + col_o<QT>(t), tmem + col_s<QT>(t) + kk * 8, bdesc, idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         return true;
       };
@@ -492,6 +501,12 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
             pk[c / 2] = pack2(p0, p1, BF16);
           }
           tmem_st32(sc + 32 * h, pk);
+          if (h == 0) {
+            // The products over these 64 keys may start while the rest is computed.
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_half[t]);
+          }
         }
         float a0, a1, a2, a3, a4, a5, a6, a7;
         f2_unpack(acc2[0], a0, a1);
