@@ -188,10 +188,13 @@ int usp_plan_set_pack_mode(usp_plan* plan, int32_t mode);
  * first Q K^T under the previous item's last key tiles. Automatic mode uses
  * one CTA per SM when an item has at most 16 key tiles of 256 (short
  * sequences, where a CTA's fixed costs are a large share), and one CTA per
- * item otherwise. A cap below the SM count leaves SMs to kernels running
- * beside the block on other streams. Results do not depend on it (each item
- * is computed the same way). The fp32 path ignores it. Errors:
- * USP_ERR_INVALID_ARG for max_ctas < 0.
+ * item otherwise. Under a cap (and with USP_ATTN_AUTO) the launch takes the
+ * one-tile kernel; the USP_ATTN_TWO_CTA kernel, chosen explicitly, walks its
+ * items with the cap's CTA count instead of two per SM; the
+ * USP_ATTN_TWO_TILE kernel ignores the cap. A cap below the SM count leaves
+ * SMs to kernels running beside the block on other streams. Results do not
+ * depend on it (each item is computed the same way). The fp32 path ignores
+ * it. Errors: USP_ERR_INVALID_ARG for max_ctas < 0.
  */
 int usp_plan_set_attention_ctas(usp_plan* plan, int32_t max_ctas);
 

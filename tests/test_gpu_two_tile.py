@@ -74,10 +74,11 @@ def _out64(t, w):
     return t.double().cpu().numpy() if w.dtype == "fp16" else to_f64(t, w.dtype)
 
 
-def _run(usp, w, kernel, num_chunks, ring=1, lse=None):
+def _run(usp, w, kernel, num_chunks, ring=1, lse=None, ctas=0):
     plan = usp.Plan(w.batch, w.seq_len, w.heads, w.head_dim, w.world, w.dtype, w.prefix, kv_heads=w.heads_kv,
                     ring_size=ring)
     plan.set_attention_kernel(kernel)
+    plan.set_attention_ctas(ctas)
     storage = _storage(w)
     shards = [usp.scatter_sequence(plan, _dev(x, w)) for x in storage]
     out = plan.empty_seq_shards(fill=float("nan"))
@@ -167,6 +168,32 @@ def test_two_cta_ring_matches_oracle(usp, case):
     for r in range(plan.world):
         assert_close(_out64(out[r], w), ref[r], "bf16", f"{w.name} rank={r}")
     plan.close()
+
+
+@pytest.mark.parametrize("w", TWO_CTA_CASES[:3] + TWO_CTA_CASES[-2:], ids=lambda w: w.name)
+def test_two_cta_walk_is_bit_identical(usp, w):
+    """Capped so that each CTA walks several items (item hand-off through
+    q_empty and o_free): the same bits as one item per CTA."""
+    _, p0, base = _run(usp, w, "two_cta", 1, ctas=1 << 20)
+    bits = [o.view(torch.int16).cpu() for o in base]
+    p0.close()
+    for ctas in (1, 2, 5):
+        _, pc, out = _run(usp, w, "two_cta", 1, ctas=ctas)
+        for r, o in enumerate(out):
+            assert torch.equal(o.view(torch.int16).cpu(), bits[r]), f"ctas={ctas} rank={r}"
+        pc.close()
+
+
+@pytest.mark.parametrize("case", [c for c in RING_CASES if c[0].head_dim in (64, 80)], ids=lambda c: c[0].name)
+def test_two_cta_ring_walk_is_bit_identical(usp, case):
+    w, ring = case
+    _, p0, base = _run(usp, w, "two_cta", 1, ring=ring, ctas=1 << 20)
+    bits = [o.view(torch.int16).cpu() for o in base]
+    p0.close()
+    _, pc, out = _run(usp, w, "two_cta", 1, ring=ring, ctas=3)
+    for r, o in enumerate(out):
+        assert torch.equal(o.view(torch.int16).cpu(), bits[r]), f"rank={r}"
+    pc.close()
 
 
 def test_two_cta_agrees_bitwise_with_two_tile(usp):

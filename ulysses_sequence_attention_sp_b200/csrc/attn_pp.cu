@@ -416,6 +416,99 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
     const uint32_t oc = lane_addr + col_o<QT>(t);
     const float sl2 = p.scale_log2;
     const bool tr0 = quarter == 0 && lane == 0;
+    // Epilogue of the CTA's k-th item `it` (running maximum m, denominator l):
+    // O of this tile, normalised, to the rows' destinations. Returns false if
+    // a wait gave up.
+    auto epilogue = [&](int it, int k, float m, float l) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], k & 1, abort_flag, &g_pp_error, 52 + t,
+                                             kWaitLimitNs)))
+        return false;
+      tc_fence_after();
+      if (QT == 1 && tr0) PP_TRACE(12, k);
+      // The whole row of O in one round of TMEM loads; then O may be overwritten.
+      uint32_t o[D];
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) tmem_ld16(oc + c * 16, *reinterpret_cast<uint32_t(*)[16]>(o + c * 16));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_free[t]);
+      const float inv_l = 1.f / l;
+      const PpItem w = pp_item(p, it, QT, RING);
+      const int tr = w.row0 + t * kRows + row;  // row of the full sequence
+      const bool row_ok = tr < w.q_end;
+      if (p.lse != nullptr && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
+        const int64_t li = (static_cast<int64_t>(w.hm) * p.batch + w.b) * T + tr;
+        if (in_bounds(li, 1, p.lse_ext, 22, &g_pp_bounds)) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
+      }
+      const AttnOut& out = p.out;
+      int seg_lo = 0, seg_hi = 0;
+      int64_t row_in_seg = 0;
+      if (row_ok) {
+        if (tr < out.prefix) {  // a replicated prefix row goes to every segment
+          seg_lo = 0;
+          seg_hi = out.nseg;
+          row_in_seg = tr;
+        } else {
+          const int64_t tok = tr - out.prefix;
+          int sg = 0;
+          while (sg + 1 < out.nseg && tok >= out.seg_start[sg + 1]) ++sg;
+          seg_lo = sg;
+          seg_hi = sg + 1;
+          row_in_seg = out.prefix + tok - out.seg_start[sg];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < D / 2; ++i)
+        o[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, BF16);
+      // This row's destination in segment sg (null: out of range).
+      auto row_dst = [&](int sg) -> uint16_t* {
+        const int64_t rows_s = out.prefix + out.seg_len[sg];
+        const int64_t elem =
+            ((static_cast<int64_t>(w.b) * rows_s + row_in_seg) * out.out_heads + w.hm - out.head_base) * D;
+        if (!in_bounds(elem, D, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds))
+          return nullptr;
+        return static_cast<uint16_t*>(out.seg_ptr[sg]) + elem;
+      };
+      int sg_direct = seg_lo;  // segments this thread writes itself, from its registers
+      if constexpr (QT == 1) {
+        // The warp's 32 rows, half a row per round, through its staging block:
+        // each thread writes its half row, then the warp stores the block in
+        // row-major order, consecutive threads writing consecutive 16-byte
+        // chunks of a row. The first segment goes this way; a replicated
+        // prefix row's other segments are written directly below.
+        constexpr int CH = D / 16;  // 16-byte chunks per half row
+        const uint64_t my_dst = row_ok ? reinterpret_cast<uint64_t>(row_dst(seg_lo)) : 0;
+        const uint32_t stg = smem_u32(sStg) + quarter * (32 * C::STG_STRIDE);
+        sg_direct = seg_lo + 1;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            const int i = h * (D / 4) + 4 * c;
+            st_shared_v4(stg + lane * C::STG_STRIDE + c * 16, o[i], o[i + 1], o[i + 2], o[i + 3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int st = 0; st < CH; ++st) {
+            const int q = st * 32 + lane;  // chunk q of the block: row q / CH, chunk q % CH
+            const int r = q / CH, c = q - r * CH;
+            const uint4 v = ld_shared_v4(stg + r * C::STG_STRIDE + c * 16);
+            const uint64_t d = __shfl_sync(0xffffffffu, my_dst, r);
+            if (d != 0) reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(d) + h * (D / 2))[c] = v;
+          }
+          __syncwarp();
+        }
+      }
+      for (int sg = sg_direct; sg < seg_hi; ++sg) {
+        uint4* dst = reinterpret_cast<uint4*>(row_dst(sg));
+        if (dst == nullptr) continue;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+      }
+      if (QT == 1 && tr0) PP_TRACE(13, k);
+      return true;
+    };
     bool ok = true;
     for (int it = it0, k = 0; ok && it < it_end; it += it_step, ++k) {
       if constexpr (QT == 2) k = 0;
@@ -528,96 +621,7 @@ __global__ void __launch_bounds__(pp_threads(QT), 3 - QT) attn_pp_kernel(const _
         }
       }
       if (!ok) break;
-      // Epilogue: O of this tile, normalised, to the rows' destinations.
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], k & 1, abort_flag, &g_pp_error, 52 + t,
-                                             kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (QT == 1 && tr0) PP_TRACE(12, k);
-      // The whole row of O in one round of TMEM loads; then O may be overwritten.
-      uint32_t o[D];
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) tmem_ld16(oc + c * 16, *reinterpret_cast<uint32_t(*)[16]>(o + c * 16));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->o_free[t]);
-      const float inv_l = 1.f / l;
-      const PpItem w = pp_item(p, it, QT, RING);
-      const int tr = w.row0 + t * kRows + row;  // row of the full sequence
-      const bool row_ok = tr < w.q_end;
-      if (p.lse != nullptr && row_ok) {  // sum_j exp(scale s_j) = 2^m * l
-        const int64_t li = (static_cast<int64_t>(w.hm) * p.batch + w.b) * T + tr;
-        if (in_bounds(li, 1, p.lse_ext, 22, &g_pp_bounds)) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
-      }
-      const AttnOut& out = p.out;
-      int seg_lo = 0, seg_hi = 0;
-      int64_t row_in_seg = 0;
-      if (row_ok) {
-        if (tr < out.prefix) {  // a replicated prefix row goes to every segment
-          seg_lo = 0;
-          seg_hi = out.nseg;
-          row_in_seg = tr;
-        } else {
-          const int64_t tok = tr - out.prefix;
-          int sg = 0;
-          while (sg + 1 < out.nseg && tok >= out.seg_start[sg + 1]) ++sg;
-          seg_lo = sg;
-          seg_hi = sg + 1;
-          row_in_seg = out.prefix + tok - out.seg_start[sg];
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < D / 2; ++i)
-        o[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, BF16);
-      // This row's destination in segment sg (null: out of range).
-      auto row_dst = [&](int sg) -> uint16_t* {
-        const int64_t rows_s = out.prefix + out.seg_len[sg];
-        const int64_t elem =
-            ((static_cast<int64_t>(w.b) * rows_s + row_in_seg) * out.out_heads + w.hm - out.head_base) * D;
-        if (!in_bounds(elem, D, static_cast<int64_t>(p.batch) * rows_s * out.out_heads * D, 23, &g_pp_bounds))
-          return nullptr;
-        return static_cast<uint16_t*>(out.seg_ptr[sg]) + elem;
-      };
-      int sg_direct = seg_lo;  // segments this thread writes itself, from its registers
-      if constexpr (QT == 1) {
-        // The warp's 32 rows, half a row per round, through its staging block:
-        // each thread writes its half row, then the warp stores the block in
-        // row-major order, consecutive threads writing consecutive 16-byte
-        // chunks of a row. The first segment goes this way; a replicated
-        // prefix row's other segments are written directly below.
-        constexpr int CH = D / 16;  // 16-byte chunks per half row
-        const uint64_t my_dst = row_ok ? reinterpret_cast<uint64_t>(row_dst(seg_lo)) : 0;
-        const uint32_t stg = smem_u32(sStg) + quarter * (32 * C::STG_STRIDE);
-        sg_direct = seg_lo + 1;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            const int i = h * (D / 4) + 4 * c;
-            st_shared_v4(stg + lane * C::STG_STRIDE + c * 16, o[i], o[i + 1], o[i + 2], o[i + 3]);
-          }
-          __syncwarp();
-#pragma unroll
-          for (int st = 0; st < CH; ++st) {
-            const int q = st * 32 + lane;  // chunk q of the block: row q / CH, chunk q % CH
-            const int r = q / CH, c = q - r * CH;
-            const uint4 v = ld_shared_v4(stg + r * C::STG_STRIDE + c * 16);
-            const uint64_t d = __shfl_sync(0xffffffffu, my_dst, r);
-            if (d != 0) reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(d) + h * (D / 2))[c] = v;
-          }
-          __syncwarp();
-        }
-      }
-      for (int sg = sg_direct; sg < seg_hi; ++sg) {
-        uint4* dst = reinterpret_cast<uint4*>(row_dst(sg));
-        if (dst == nullptr) continue;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-      }
-      if (QT == 1 && tr0) PP_TRACE(13, k);
+      ok = epilogue(it, k, m, l);
     }
   }
 
@@ -665,10 +669,11 @@ int launch_pp_d(const AttnLaunch& L, cudaStream_t stream) {
   const int64_t items = static_cast<int64_t>(p.q_pair_prefix[p.n_qgroups]) * L.batch * L.n_heads;
   if (items > INT32_MAX) return set_error(USP_ERR_UNSUPPORTED, "attention: %lld query tiles in one launch", (long long)items);
   p.n_items = static_cast<int32_t>(items);
-  // Two query tiles: one CTA per item. One query tile: two CTAs per SM walk
-  // the items, each starting an item's loads and first Q K^T under the end of
-  // the one before.
-  const int64_t ctas = QT == 2 ? items : std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
+  // Two query tiles: one CTA per item. One query tile: two CTAs per SM (or
+  // the caller's cap) walk the items, each starting an item's loads and first
+  // Q K^T under the end of the one before.
+  const int64_t walkers = L.max_ctas > 0 ? L.max_ctas : 2 * static_cast<int64_t>(sm_count());
+  const int64_t ctas = QT == 2 ? items : std::min<int64_t>(items, walkers);
   const dim3 grid(static_cast<unsigned>(ctas));
   if (ring)
     attn_pp_kernel<D, QT, BF16, true><<<grid, pp_threads(QT), C::SMEM_BYTES, stream>>>(p);
