@@ -1,5 +1,6 @@
-// Non-causal softmax attention on the tcgen05 tensor cores, two query tiles
-// per CTA ("ping-pong").
+// Non-causal softmax attention on the tcgen05 tensor cores with 128-key
+// tiles: two query tiles per CTA ("ping-pong", QT = 2), or one query tile per
+// CTA with two CTAs per SM (QT = 1).
 //
 // What it computes is exactly what attn_tc.cu computes (API page
 // "mstar.model.components.distributed.sequence_parallel", ulysses_attention /
@@ -11,25 +12,31 @@
 // exchange, fused), with the Ulysses + Ring key-block walk (RING) and
 // grouped-query attention as in attn_tc.cu.
 //
-// How it is organised differs. One CTA takes two 128-row query tiles A and B
-// of one (batch, head) and walks the keys in tiles of 128:
-//   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread
-//               per query row (TMEM lane = row), holding the row's 128 scores,
-//               so no partial maxima are exchanged between threads
-//   warp 8      TMA producer: Q_A and Q_B once, then K and V tiles into rings
-//   warp 9      TMEM allocator and MMA issuer (one thread), in the order
-//                 S_A(0) S_B(0) | PV_A(j-1) S_A(j) PV_B(j-1) S_B(j) | ...
-//               so that while the softmax of one tile runs, the tensor core
-//               works on the other tile's products.
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
+// How it is organised differs. A work item is QT 128-row query tiles of one
+// (batch, head); a CTA walks the keys of its item in tiles of 128:
+//   warps 0..4QT-1  softmax, four warps per tile: one thread per query row
+//                   (TMEM lane = row), holding the row's 128 scores, so no
+//                   partial maxima are exchanged between threads
+//   warp 4QT        TMA producer: the item's Q tiles, then K and V tiles into rings
+//   warp 4QT+1      TMEM allocator and MMA issuer (one thread), in the order
+//                     S_A(0) S_B(0) | PV_A(j-1) S_A(j) PV_B(j-1) S_B(j) | ...
+//                   (tile B only when QT = 2), so that while the softmax of one
+//                   tile runs, the tensor core works on the other tile's products
+//                   (with QT = 1, on the other CTA's).
+// TMEM columns: S of tile t at 128t, O of tile t at 128 QT + 128t (D wide).
 // P (128 keys, two 16-bit values per column) is written over the first 64
-// columns of its tile's S, which the softmax has already read into registers;
-// the next S of that tile is issued only after the P.V that reads P, and the
-// tensor core runs one thread's MMAs in issue order.
+// columns of its tile's S, which the softmax has already read into registers,
+// in two halves; the P.V products over the first half's 64 keys are issued as
+// soon as that half is stored. The next S of that tile is issued only after
+// the P.V that reads P, and the tensor core runs one thread's MMAs in order.
 // O is rescaled in TMEM only when a row maximum grows by more than 2^8 (the
 // stale maximum is kept otherwise: exact, since numerator and denominator use
 // the same maximum). A tile's O is only ever written by its own P.V, which
 // has completed whenever the tile's next S has (one commit covers both).
+// QT = 2 launches one CTA per item. QT = 1 launches two CTAs per SM that walk
+// the items; every ring stage and barrier phase follows the CTA's running tile
+// count, an item's Q loads once the previous item's last S is done (q_empty),
+// and its first P.V waits for the previous epilogue's reads of O (o_free).
 #include <algorithm>
 #include <cmath>
 
