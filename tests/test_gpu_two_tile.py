@@ -207,10 +207,11 @@ def test_two_cta_agrees_bitwise_with_two_tile(usp):
     p2.close()
 
 
-def test_two_tile_lse(usp):
+@pytest.mark.parametrize("kernel", ["two_tile", "two_cta"])
+def test_two_tile_lse(usp, kernel):
     w = CASES[1]
     lse = torch.full((w.heads, w.batch, w.tokens), float("nan"), dtype=torch.float32, device="cuda")
-    storage, plan, _ = _run(usp, w, "two_tile", 1, lse=lse)
+    storage, plan, _ = _run(usp, w, kernel, 1, lse=lse)
     q, k, _v = (_f64(x, w) for x in storage)
     scale = 1.0 / np.sqrt(w.head_dim)
     got = lse.cpu().numpy()
