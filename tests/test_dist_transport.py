@@ -1,4 +1,4 @@
-"""The multi-process transport's host logic on CPU ranks (gloo, world 2 and 3).
+"""The multi-process transport's host logic on CPU ranks (gloo, world 2, 3 and 4).
 
 One process per rank. Each rank builds its send blocks by the wire format the
 header states (per-peer blocks of the chunk's heads for the all-to-all form,
@@ -32,6 +32,8 @@ CASES = [
     (1, 37, 6, 6, 8, 2, 0, (1, 2, 4)),
     (2, 37, 6, 3, 4, 3, 1, (1, 2, 3)),   # grouped-query (2 q heads per kv head), cls prefix
     (1, 40, 7, 7, 4, 3, 1, (1, 2)),      # ragged heads 3,2,2; chunks 2,1 then 2,0
+    (1, 29, 10, 10, 4, 4, 1, (1, 3)),    # four ranks: tokens 8,7,7,7, heads 3,3,2,2, cls prefix
+    (2, 33, 8, 4, 8, 4, 0, (1, 2)),      # four ranks, grouped-query (one kv head per rank)
 ]
 
 
