@@ -50,8 +50,9 @@ __device__ uint32_t g_pp_error;   // first wait that ran out (site code), 0 if n
 __device__ uint32_t g_pp_bounds;  // bounds-checking builds: first out-of-range site, 0 if none
 
 // Pipeline trace (built only with -DUSP_TRACE): clock64() at pipeline events
-// of one CTA (query tile group min(7, half the groups), batch-head min(3, last)),
-// [event][key tile]; read with usp_debug_read_trace_pp.
+// of one CTA (CTA min(7, half the grid); the grid is one-dimensional, so the
+// second condition always holds), [event][the CTA's key tile, or item for the
+// per-item stamps]; read with usp_debug_read_trace_pp.
 #ifdef USP_TRACE
 constexpr int kPpTraceEvents = 16, kPpTraceTiles = 256;
 __device__ unsigned long long g_pp_trace[kPpTraceEvents][kPpTraceTiles];
